@@ -1,0 +1,376 @@
+// C ABI of libslim.so (declared in include/slim.h): argument checks,
+// workspace carve-up, kernel selection and the measured ordering table.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <map>
+#include <mutex>
+#include <tuple>
+#include <vector>
+
+#include "slim_internal.h"
+
+namespace slim {
+
+// ---------------------------------------------------------------------------- device queries
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    return 148;  // B200
+  }
+  return n;
+}
+
+int max_smem_optin() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    return 232448;  // B200: 227 KiB
+  }
+  return n;
+}
+
+// ---------------------------------------------------------------------------- tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                         uint32_t box_inner, uint32_t box_outer, bool swizzle128) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------- workspace
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+size_t esize(int dtype) { return dtype == SLIM_BF16 ? 2 : 4; }
+
+struct WsLayout {
+  size_t U, m, l, meta, vbuf, stage, total;
+  int max_items;
+};
+
+WsLayout ws_layout(int dtype, int B, int d, int H, int64_t cap, int variant) {
+  WsLayout w{};
+  const int items = std::max(num_sms(), B);
+  w.max_items = items;
+  const bool need_b = variant != SLIM_VARIANT_A;
+  const bool need_a = variant != SLIM_VARIANT_B;
+  size_t u_floats = 0;
+  if (need_b) u_floats = std::max(u_floats, static_cast<size_t>(items) * H * d);
+  if (need_a) u_floats = std::max(u_floats, static_cast<size_t>(items) * d);
+  size_t o = 0;
+  w.U = o;
+  o += up(u_floats * 4);
+  w.m = o;
+  o += up(static_cast<size_t>(items) * H * 4);
+  w.l = o;
+  o += up(static_cast<size_t>(items) * H * 4);
+  w.meta = o;
+  o += up(meta_ints(B) * 4);
+  w.vbuf = o;
+  if (need_a) o += up(static_cast<size_t>(B) * cap * d * esize(dtype));
+  w.stage = o;
+  o += up(static_cast<size_t>(B) * d * 4) * 2 + up(static_cast<size_t>(B) * d * esize(dtype));
+  w.total = o;
+  return w;
+}
+
+SplitWorkspace carve(void* base, const WsLayout& w) {
+  char* c = static_cast<char*>(base);
+  SplitWorkspace s;
+  s.U = reinterpret_cast<float*>(c + w.U);
+  s.m = reinterpret_cast<float*>(c + w.m);
+  s.l = reinterpret_cast<float*>(c + w.l);
+  s.meta = reinterpret_cast<int32_t*>(c + w.meta);
+  s.vbuf = c + w.vbuf;
+  s.qstage = c + w.stage;
+  s.max_items = w.max_items;
+  return s;
+}
+
+thread_local int g_last_launches = 0;
+
+// ---------------------------------------------------------------------------- ordering table
+struct TuneKey {
+  int dtype, B, d, H;
+  bool operator<(const TuneKey& o) const {
+    return std::tie(dtype, B, d, H) < std::tie(o.dtype, o.B, o.d, o.H);
+  }
+};
+struct TunePoint {
+  int64_t T;
+  float ms_a, ms_b;
+};
+std::mutex g_tune_mu;
+std::map<TuneKey, std::vector<TunePoint>> g_tune;
+
+bool valid_dims(int dtype, int B, int d, int H, int64_t cap) {
+  return (dtype == SLIM_F32 || dtype == SLIM_BF16) && B >= 1 && d >= 1 && H >= 1 && d % H == 0 && cap >= 1 &&
+         cap <= (int64_t(1) << 31) - 1 && static_cast<int64_t>(B) * cap <= (int64_t(1) << 31) - 1;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+}  // namespace
+
+cudaError_t launch_prefill_simt(const void* X, const void* W, void* kcache, const int32_t* lens, int dtype, int B,
+                                int n, int d, int64_t cap, cudaStream_t st, int* launches);
+cudaError_t launch_prefill_tc(const void* X, const void* W, void* kcache, const int32_t* lens, int B, int n, int d,
+                              int64_t cap, cudaStream_t st, int* launches);
+cudaError_t launch_rows_gemm_tc(const void* A, const void* W, void* Y, const int32_t* lens, int rows_extra, int B,
+                                int d, int64_t cap, cudaStream_t st, int* launches);
+bool gemm_tc_supported(int d);
+cudaError_t launch_advance_lens(int32_t* lens, int B, int n, int64_t cap, int32_t* status, cudaStream_t st,
+                                int* launches);
+
+cudaError_t launch_rows_gemm_any(const void* A, const void* W, void* Y, const int32_t* lens, int rows_extra,
+                                 int dtype, int B, int d, int64_t cap, cudaStream_t st, int* launches) {
+  if (dtype == SLIM_BF16 && gemm_tc_supported(d))
+    return launch_rows_gemm_tc(A, W, Y, lens, rows_extra, B, d, cap, st, launches);
+  return launch_rows_gemm(A, W, Y, lens, rows_extra, dtype, B, d, cap, st, launches);
+}
+
+}  // namespace slim
+
+using namespace slim;
+
+// ============================================================================ C ABI
+extern "C" {
+
+int slim_version(void) { return 100; }
+
+int slim_last_launch_count(void) { return g_last_launches; }
+
+const char* slim_strerror(int code) {
+  switch (code) {
+    case SLIM_OK: return "success";
+    case SLIM_EINVAL: return "invalid argument (null pointer, size, d % H, dtype or variant)";
+    case SLIM_EWORKSPACE: return "workspace missing, too small or not 256-byte aligned";
+    case SLIM_ECUDA: return "CUDA runtime or launch failure";
+    case SLIM_EUNSUPPORTED: return "no kernel for this shape/dtype";
+    case SLIM_DEV_OVERFLOW: return "device: append would exceed cache capacity (sequence skipped)";
+    case SLIM_DEV_BADLEN: return "device: length outside [0, cap] (sequence skipped)";
+    case SLIM_DEV_TIMEOUT: return "device: a bounded wait gave up (internal error)";
+    default: break;
+  }
+  if (code > 0 && code < 8) return "device: several status bits set";
+  return "unknown code";
+}
+
+int slim_prefill_k(const void* X, const void* W_K, void* Kcache, int32_t* lens, int dtype, int B, int n, int d,
+                   int64_t cap, int32_t* dev_status, void* stream) {
+  if (!X || !W_K || !Kcache || !lens || !dev_status || n < 1) return SLIM_EINVAL;
+  if (!valid_dims(dtype, B, d, 1, cap)) return SLIM_EINVAL;
+  if (static_cast<int64_t>(n) > cap) return SLIM_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int launches = 0;
+  cudaError_t e;
+  if (dtype == SLIM_BF16 && gemm_tc_supported(d) && aligned(X, 16) && aligned(W_K, 16) && aligned(Kcache, 16))
+    e = launch_prefill_tc(X, W_K, Kcache, lens, B, n, d, cap, st, &launches);
+  else
+    e = launch_prefill_simt(X, W_K, Kcache, lens, dtype, B, n, d, cap, st, &launches);
+  if (e == cudaSuccess) e = launch_advance_lens(lens, B, n, cap, dev_status, st, &launches);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return e == cudaErrorNotSupported ? SLIM_EUNSUPPORTED : SLIM_ECUDA;
+  }
+  g_last_launches = launches;
+  return SLIM_OK;
+}
+
+size_t slim_decode_workspace_bytes(int dtype, int B, int d, int H, int64_t cap, int variant) {
+  if (!valid_dims(dtype, B, d, H, cap) || variant < SLIM_AUTO || variant > SLIM_VARIANT_B) return 0;
+  return ws_layout(dtype, B, d, H, cap, variant).total;
+}
+
+int slim_select_variant(int dtype, int B, int d, int H, int64_t T) {
+  std::lock_guard<std::mutex> g(g_tune_mu);
+  auto it = g_tune.find(TuneKey{dtype, B, d, H});
+  if (it == g_tune.end() || it->second.empty() || T < 1) return SLIM_VARIANT_B;
+  const TunePoint* best = nullptr;
+  double bestd = 0;
+  for (const auto& p : it->second) {
+    const double dist = std::fabs(std::log(static_cast<double>(p.T)) - std::log(static_cast<double>(T)));
+    if (!best || dist < bestd) {
+      best = &p;
+      bestd = dist;
+    }
+  }
+  return (best->ms_a < best->ms_b) ? SLIM_VARIANT_A : SLIM_VARIANT_B;
+}
+
+int slim_tune_record(int dtype, int B, int d, int H, int64_t T, float ms_a, float ms_b) {
+  if (!valid_dims(dtype, B, d, H, T) || !(ms_a > 0.f) || !(ms_b > 0.f)) return SLIM_EINVAL;
+  std::lock_guard<std::mutex> g(g_tune_mu);
+  auto& v = g_tune[TuneKey{dtype, B, d, H}];
+  for (auto& p : v)
+    if (p.T == T) {
+      p.ms_a = ms_a;
+      p.ms_b = ms_b;
+      return SLIM_OK;
+    }
+  v.push_back(TunePoint{T, ms_a, ms_b});
+  return SLIM_OK;
+}
+
+void slim_tune_clear(void) {
+  std::lock_guard<std::mutex> g(g_tune_mu);
+  g_tune.clear();
+}
+
+int slim_decode_step(const float* q, const void* k_new, void* Kcache, int32_t* lens, const void* W_KV, int dtype,
+                     int B, int d, int H, int64_t cap, int variant, int64_t t_hint, float* out, void* workspace,
+                     size_t ws_bytes, int32_t* dev_status, void* stream) {
+  if (!q || !Kcache || !lens || !W_KV || !out || !dev_status) return SLIM_EINVAL;
+  if (!valid_dims(dtype, B, d, H, cap) || variant < SLIM_AUTO || variant > SLIM_VARIANT_B) return SLIM_EINVAL;
+  if (!aligned(q, 16) || !aligned(Kcache, 16) || (k_new && !aligned(k_new, 16)) || !aligned(W_KV, 16))
+    return SLIM_EINVAL;
+  if ((static_cast<size_t>(d) * esize(dtype)) % 16 != 0) return SLIM_EUNSUPPORTED;
+  if (!workspace || !aligned(workspace, kAlign)) return SLIM_EWORKSPACE;
+  const WsLayout wl = ws_layout(dtype, B, d, H, cap, variant);
+  if (ws_bytes < wl.total) return SLIM_EWORKSPACE;
+  int v = variant;
+  if (v == SLIM_AUTO) v = slim_select_variant(dtype, B, d, H, t_hint > 0 ? t_hint : cap);
+
+  DecodeArgs a{q, k_new, Kcache, lens, W_KV, dtype, B, d, H, cap, out, dev_status};
+  SplitWorkspace ws = carve(workspace, wl);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int launches = 0;
+  cudaError_t e = cudaSuccess;
+  if (v == SLIM_VARIANT_B) {
+    bool tc = false;
+    if (dtype == SLIM_BF16 && decode_b_tc_supported(B, d, H)) {
+      e = launch_decode_b_tc(a, ws, st, &launches);
+      tc = (e == cudaSuccess);
+      if (e == cudaErrorNotSupported) e = cudaSuccess;
+    }
+    if (!tc && e == cudaSuccess) {
+      if (!decode_b_simt_supported(B, d, H)) return SLIM_EUNSUPPORTED;
+      e = launch_decode_b_simt(a, ws, st, &launches);
+    }
+    if (e == cudaSuccess) e = launch_reduce_b(a, ws, /*pdl=*/true, st, &launches);
+  } else {
+    if (!decode_a_supported(dtype, B, d, H)) return SLIM_EUNSUPPORTED;
+    e = launch_decode_a(a, ws, st, &launches);
+  }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return e == cudaErrorNotSupported ? SLIM_EUNSUPPORTED : SLIM_ECUDA;
+  }
+  g_last_launches = launches;
+  return SLIM_OK;
+}
+
+int slim_decode_step_host(const float* q_host, const void* k_new_host, void* Kcache, int32_t* lens,
+                          const void* W_KV, int dtype, int B, int d, int H, int64_t cap, int variant, int64_t t_hint,
+                          float* out_host, void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream) {
+  if (!q_host || !out_host) return SLIM_EINVAL;
+  if (!valid_dims(dtype, B, d, H, cap)) return SLIM_EINVAL;
+  if (!workspace || !aligned(workspace, kAlign)) return SLIM_EWORKSPACE;
+  const WsLayout wl = ws_layout(dtype, B, d, H, cap, variant);
+  if (ws_bytes < wl.total) return SLIM_EWORKSPACE;
+  char* stage = static_cast<char*>(workspace) + wl.stage;
+  const size_t qb = static_cast<size_t>(B) * d * 4, kb = static_cast<size_t>(B) * d * esize(dtype);
+  float* q_dev = reinterpret_cast<float*>(stage);
+  float* out_dev = reinterpret_cast<float*>(stage + up(qb));
+  void* k_dev = stage + 2 * up(qb);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(q_dev, q_host, qb, cudaMemcpyHostToDevice, st) != cudaSuccess) {
+    cudaGetLastError();
+    return SLIM_ECUDA;
+  }
+  if (k_new_host && cudaMemcpyAsync(k_dev, k_new_host, kb, cudaMemcpyHostToDevice, st) != cudaSuccess) {
+    cudaGetLastError();
+    return SLIM_ECUDA;
+  }
+  const int r = slim_decode_step(q_dev, k_new_host ? k_dev : nullptr, Kcache, lens, W_KV, dtype, B, d, H, cap,
+                                 variant, t_hint, out_dev, workspace, ws_bytes, dev_status, stream);
+  if (r != SLIM_OK) return r;
+  if (cudaMemcpyAsync(out_host, out_dev, qb, cudaMemcpyDeviceToHost, st) != cudaSuccess) {
+    cudaGetLastError();
+    return SLIM_ECUDA;
+  }
+  return SLIM_OK;
+}
+
+int slim_tune(const float* q, void* Kcache, int32_t* lens, const int32_t* lens_restore_host, const void* W_KV,
+              int dtype, int B, int d, int H, int64_t cap, const int64_t* Ts, int nT, int reps, float* out,
+              void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream) {
+  if (!Ts || nT < 1 || reps < 1 || !lens_restore_host) return SLIM_EINVAL;
+  if (!valid_dims(dtype, B, d, H, cap)) return SLIM_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  std::vector<int32_t> lv(static_cast<size_t>(B));
+  cudaEvent_t e0, e1;
+  if (cudaEventCreate(&e0) != cudaSuccess || cudaEventCreate(&e1) != cudaSuccess) return SLIM_ECUDA;
+  int rc = SLIM_OK;
+  for (int i = 0; i < nT && rc == SLIM_OK; ++i) {
+    if (Ts[i] < 1 || Ts[i] > cap) {
+      rc = SLIM_EINVAL;
+      break;
+    }
+    std::fill(lv.begin(), lv.end(), static_cast<int32_t>(Ts[i]));
+    if (cudaMemcpyAsync(lens, lv.data(), lv.size() * 4, cudaMemcpyHostToDevice, st) != cudaSuccess) {
+      rc = SLIM_ECUDA;
+      break;
+    }
+    float ms[2] = {0.f, 0.f};
+    const int vars[2] = {SLIM_VARIANT_A, SLIM_VARIANT_B};
+    for (int k = 0; k < 2 && rc == SLIM_OK; ++k) {
+      rc = slim_decode_step(q, nullptr, Kcache, lens, W_KV, dtype, B, d, H, cap, vars[k], 0, out, workspace,
+                            ws_bytes, dev_status, stream);  // warm-up
+      if (rc != SLIM_OK) break;
+      cudaEventRecord(e0, st);
+      for (int r = 0; r < reps && rc == SLIM_OK; ++r)
+        rc = slim_decode_step(q, nullptr, Kcache, lens, W_KV, dtype, B, d, H, cap, vars[k], 0, out, workspace,
+                              ws_bytes, dev_status, stream);
+      cudaEventRecord(e1, st);
+      if (cudaEventSynchronize(e1) != cudaSuccess) rc = SLIM_ECUDA;
+      cudaEventElapsedTime(&ms[k], e0, e1);
+      ms[k] /= reps;
+    }
+    if (rc == SLIM_OK) slim_tune_record(dtype, B, d, H, Ts[i], ms[0], ms[1]);
+  }
+  if (cudaMemcpyAsync(lens, lens_restore_host, static_cast<size_t>(B) * 4, cudaMemcpyHostToDevice, st) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess)
+    rc = SLIM_ECUDA;
+  cudaEventDestroy(e0);
+  cudaEventDestroy(e1);
+  cudaGetLastError();
+  return rc;
+}
+
+}  // extern "C"

@@ -1,0 +1,84 @@
+// Internal declarations shared by the libslim translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/slim.h"
+
+namespace slim {
+
+// Bounded spin: ~16M polls with a 64 ns back-off ≈ 1-2 s before a wait gives up.
+constexpr uint32_t kWaitSpinLimit = 1u << 24;
+
+// Work-list metadata written by the split kernel for the merge kernel:
+//   meta[0]          total number of work items
+//   meta[1 + b]      first item of sequence b (b = 0..B), meta[1 + B] = total
+//   meta[2 + B + b]  flags of sequence b (kSeqAppend: lens[b] must advance by one)
+constexpr int kSeqAppend = 1;
+__host__ __device__ inline size_t meta_ints(int B) { return static_cast<size_t>(2 * B + 2); }
+
+// Scratch of the split-T orderings, carved from the caller's workspace.
+struct SplitWorkspace {
+  float* U;      // (b): [items][H][d] unnormalised softmax·K rows;  (a): [items][d] softmax·V
+  float* m;      // [items][H] running max (log2 domain)
+  float* l;      // [items][H] softmax denominators relative to m
+  int32_t* meta; // meta_ints(B)
+  void* vbuf;    // (a) only: [B][cap][d] materialised V = K·W_KV
+  void* qstage;  // staging for slim_decode_step_host: q, k_new, out
+  int max_items;
+};
+
+struct DecodeArgs {
+  const float* q;
+  const void* k_new;
+  void* kcache;
+  int32_t* lens;
+  const void* w_kv;
+  int dtype, B, d, H;
+  int64_t cap;
+  float* out;
+  int32_t* status;
+};
+
+// Split decomposition of the attended rows into work items; computed the
+// same way on the device by every CTA of a split kernel.
+struct SplitPlan {
+  int n_slots;   // clusters (work slots) launched
+  int min_rows;  // smallest chunk worth its partial write
+};
+
+// ---- launchers (return cudaError_t of the launch) ----
+// Variant (b), tcgen05 path (bf16). Returns cudaErrorNotSupported if the shape has no tcgen05 config.
+cudaError_t launch_decode_b_tc(const DecodeArgs& a, const SplitWorkspace& ws, cudaStream_t st, int* launches);
+bool decode_b_tc_supported(int B, int d, int H);
+// Variant (b), CUDA-core path (fp32 or bf16 cache).
+cudaError_t launch_decode_b_simt(const DecodeArgs& a, const SplitWorkspace& ws, cudaStream_t st, int* launches);
+bool decode_b_simt_supported(int B, int d, int H);
+// Merge of variant (b) partials and the W_KV projection; advances lens.
+cudaError_t launch_reduce_b(const DecodeArgs& a, const SplitWorkspace& ws, bool pdl, cudaStream_t st,
+                            int* launches);
+// Variant (a): append, V = K·W_KV, split flash-decode over K and V, merge.
+cudaError_t launch_decode_a(const DecodeArgs& a, const SplitWorkspace& ws, cudaStream_t st, int* launches);
+bool decode_a_supported(int dtype, int B, int d, int H);
+// Prompt-phase projection K = X·W_K into the cache at lens[b]; then lens += n.
+cudaError_t launch_prefill(const void* X, const void* W, void* kcache, int32_t* lens, int dtype, int B, int n, int d,
+                           int64_t cap, int32_t* status, cudaStream_t st, int* launches);
+cudaError_t launch_reduce_a(const DecodeArgs& a, const SplitWorkspace& ws, cudaStream_t st, int* launches);
+// Row-wise GEMM used by variant (a): Y[b][t] = K[b][t]·W for t < lens[b] (+append) rows of each sequence.
+// _any picks the tcgen05 kernel for bf16 shapes it supports, else the CUDA-core one.
+cudaError_t launch_rows_gemm_any(const void* A, const void* W, void* Y, const int32_t* lens, int rows_extra,
+                                 int dtype, int B, int d, int64_t cap, cudaStream_t st, int* launches);
+cudaError_t launch_rows_gemm(const void* A, const void* W, void* Y, const int32_t* lens, int rows_extra, int dtype,
+                             int B, int d, int64_t cap, cudaStream_t st, int* launches);
+
+// Tensor map encoding through the driver entry point (no link-time libcuda dependency).
+bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
+                         uint32_t box_inner, uint32_t box_outer, bool swizzle128);
+
+int num_sms();
+int max_smem_optin();
+
+}  // namespace slim

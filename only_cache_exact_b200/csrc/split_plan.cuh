@@ -1,0 +1,121 @@
+// Split-T work list for the decode kernels ("flash-decoding" style): the
+// attended rows of every sequence are cut into row chunks so that the total
+// number of chunks fills the launched work slots, then each slot (a CTA or a
+// CTA cluster) reduces one chunk to a softmax partial. Every CTA of a split
+// kernel computes the same plan from `lens`, so no pre-pass kernel is needed.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace slim {
+
+__device__ __forceinline__ long long warp_sum_ll(long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ int warp_sum_int(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+struct SplitItem {
+  int b;     // sequence, -1 if this slot has no work
+  int row0;  // first row of the chunk within the sequence
+  int row1;  // one past the last row
+  int nb;    // attended rows of the sequence (incl. the appended one)
+};
+
+// Run by ONE full warp. s_nb, s_rows: [B]; s_off: [B+1] (shared memory).
+// n_slots must be >= B so that one chunk per sequence always fits.
+// report != 0: also writes the merge metadata and ORs length errors into *status.
+__device__ inline void plan_split(const int32_t* __restrict__ lens, int B, int64_t cap, int append, int n_slots,
+                                  int min_rows, int* s_nb, int* s_rows, int* s_off, int32_t* meta, int32_t* status,
+                                  bool report) {
+  const int lane = threadIdx.x & 31;
+  int bad = 0;
+  for (int b = lane; b < B; b += 32) {
+    const int L = __ldg(lens + b);
+    int nb;
+    if (L < 0 || static_cast<int64_t>(L) > cap) {
+      nb = 0;
+      bad |= SLIM_DEV_BADLEN;
+    } else if (append && static_cast<int64_t>(L) >= cap) {
+      nb = 0;
+      bad |= SLIM_DEV_OVERFLOW;
+    } else {
+      nb = L + append;
+    }
+    s_nb[b] = nb;
+    if (report) meta[2 + B + b] = (nb > 0 && append) ? kSeqAppend : 0;
+  }
+  bad = __reduce_or_sync(0xffffffffu, bad);
+  if (report && lane == 0 && bad) atomicOr(status, bad);
+  __syncwarp();
+
+  // Smallest chunk length C (a multiple of 16 rows, at least min_rows) such
+  // that cutting every sequence into ceil(nb / C) chunks needs no more than
+  // n_slots work items: this minimises the longest chunk, i.e. the step time.
+  int max_nb = 0;
+  for (int b = lane; b < B; b += 32) max_nb = max(max_nb, s_nb[b]);
+  max_nb = __reduce_max_sync(0xffffffffu, max_nb);
+  int lo = (max(min_rows, 16) + 15) >> 4, hi = max((max_nb + 15) >> 4, lo);
+#pragma unroll 1
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    const int C = mid << 4;
+    int cnt = 0;
+    for (int b = lane; b < B; b += 32) cnt += (s_nb[b] + C - 1) / C;
+    cnt = warp_sum_int(cnt);
+    if (cnt <= n_slots) hi = mid; else lo = mid + 1;
+  }
+  const int chunk = lo << 4;
+
+  int carry = 0;
+  for (int base = 0; base < B; base += 32) {
+    const int b = base + lane;
+    int c = 0;
+    if (b < B) {
+      const int nb = s_nb[b];
+      s_rows[b] = chunk;
+      if (nb > 0) c = (nb + chunk - 1) / chunk;
+    }
+    int x = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (b < B) s_off[b] = carry + x - c;
+    carry += __shfl_sync(0xffffffffu, x, 31);
+  }
+  if (lane == 0) s_off[B] = carry;
+  __syncwarp();
+  if (report) {
+    for (int b = lane; b <= B; b += 32) meta[1 + b] = s_off[b];
+    if (lane == 0) meta[0] = carry;
+  }
+}
+
+// Work item of slot `slot` from a finished plan (any thread).
+__device__ inline SplitItem plan_lookup(int slot, int B, const int* s_nb, const int* s_rows, const int* s_off) {
+  SplitItem it{-1, 0, 0, 0};
+  if (slot >= s_off[B]) return it;
+  int lo = 0, hi = B;  // largest b with s_off[b] <= slot
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (s_off[mid] <= slot) lo = mid; else hi = mid;
+  }
+  // skip empty sequences sharing the same offset
+  int b = lo;
+  while (b < B && s_off[b + 1] <= slot) ++b;
+  const int c = slot - s_off[b];
+  it.b = b;
+  it.nb = s_nb[b];
+  it.row0 = c * s_rows[b];
+  it.row1 = min(it.row0 + s_rows[b], it.nb);
+  return it;
+}
+
+}  // namespace slim
