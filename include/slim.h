@@ -168,6 +168,20 @@ const char* slim_strerror(int code);
  * host thread enqueued. */
 int slim_last_launch_count(void);
 
+/* slim_timing_enable — measurement aid. With n > 0, every following
+ * slim_decode_step on this host thread records a pair of CUDA events
+ * (owned by the library, timing enabled) on `stream` immediately before and
+ * after its split kernel (the kernel that streams the K cache), cycling
+ * through n pairs; this also works inside CUDA-graph capture, where the
+ * records become event nodes. n = 0 destroys the events. Returns SLIM_OK,
+ * SLIM_EINVAL (n < 0) or SLIM_ECUDA. Host-side only; allocates no device memory. */
+int slim_timing_enable(int n);
+
+/* slim_timing_read — after `stream` has been synchronised, writes the
+ * elapsed milliseconds of pair i into ms[i] for i < min(n, pairs recorded)
+ * and returns that count (negative SLIM_E* on error). */
+int slim_timing_read(float* ms, int n);
+
 /* slim_version — ABI version (major*100 + minor). */
 int slim_version(void);
 

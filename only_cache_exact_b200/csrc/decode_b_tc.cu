@@ -1,4 +1,4 @@
-// Generation step, ordering (b), on tcgen05 tensor cores (bf16 K cache).
+// Generation step, ordering (b), on tensor cores (bf16 K cache).
 //
 // Slim Attention article, section "K-Cache is All You Need", generation
 // phase, second option: multiply the per-head softmax rows by K first (a full
@@ -8,28 +8,43 @@
 //     m_h = running max of the scaled scores (log2 domain)
 //     l_h = sum_t 2^(s_ht - m_h)
 //     U_h = sum_t 2^(s_ht - m_h) · K_t            (a full d-row, fp32)
-// reduce_b.cu merges the partials and applies W_KV.
+// reduce.cu merges the partials and applies W_KV.
 //
-// Per CTA (one cluster of CL CTAs per work item; CTA r owns the columns
-// [r·d/CL, (r+1)·d/CL) and the heads whose columns lie there):
-//   warp 0      TMA producer: K tile = TT rows × (d/CL) columns, 128-byte
-//               swizzled boxes of 16 rows × 64 columns, evict-first in L2.
-//   warp 1      MMA issuer: Uᵀ (d-tile of 128 × heads) += K_tileᵀ · Pᵀ with
-//               tcgen05.mma kind::f16 (A = K tile read MN-major, B = P
-//               K-major), accumulator in TMEM: lane = d column, column = head.
-//   warps 2..5  scores q_h·K_t (fp32 CUDA cores, 8 lanes per row and
-//               shuffle reduction), online softmax with a lazy max (the
-//               accumulator is rescaled in TMEM only when a head's max grows by
-//               more than 2^8), P in bf16 to shared memory (and to the peer CTA
-//               of the cluster through distributed shared memory), epilogue
-//               TMEM -> partials in global memory.
+// A cluster of CL CTAs shares one work item; CTA r owns the columns
+// [r·dS, (r+1)·dS), dS = d/CL <= 1024, and the heads whose columns lie there.
+// Per CTA (14 warps):
+//   warp 0       TMA producer: a K tile is TT rows x dS columns, one 3-D box
+//                per 16-row slab (128-byte swizzle), evict-first in L2.
+//   warp 1       MMA issuer: U[heads, own columns] += P[heads, rows] · K[rows,
+//                own columns] with tcgen05.mma kind::f16, M = 64 (heads),
+//                N <= 256 (columns), K = 16 rows; the K slab is read in place
+//                as the MN-major B operand. Two M=64 accumulators interleave in
+//                TMEM (lane offsets 0 and 16), so 1024 columns fit in the 512
+//                TMEM columns.
+//   warps 2..5   correction and epilogue: the lazy online-softmax rescale of
+//                the accumulator rows whose max grew by more than 2^8, and
+//                TMEM -> partials in global memory.
+//   warps 6..13  scores: per head, q_h·K_t for 16 rows at a time with warp
+//                mma.sync (q split into bf16 high and low parts, fp32
+//                accumulation), running max, P in bf16 to shared memory and to
+//                the other CTAs of the cluster (distributed shared memory).
 // Every mbarrier wait is bounded; a timeout sets SLIM_DEV_TIMEOUT and the
 // kernel drains its copies and MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "split_plan.cuh"
 
 namespace slim {
+
+// A head's running max may grow by this much (log2 units) before its TMEM row
+// is rescaled: P stays <= 2^8 in bf16 and no precision is lost.
+constexpr float kLazyRescaleLog2 = 8.f;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kTCThreads = (6 + kSoftmaxWarps) * 32;
+constexpr int kMaxColsPerCTA = 1024;  // two interleaved M=64 accumulators x 512 TMEM columns
+constexpr int kPRows = 64;            // M of the P·K MMA: heads, padded
 
 struct DecodeTCParams {
   const float* q;
@@ -44,9 +59,9 @@ struct DecodeTCParams {
   int B, d, H;
   int64_t cap;
   int append;
-  int n_slots;
+  int n_groups;   // clusters launched
+  int max_items;  // work items the workspace holds
   int stages;
-  int npad;
   int min_rows;
   uint32_t tmem_cols;
   float scale_log2;
@@ -54,21 +69,24 @@ struct DecodeTCParams {
 
 // Shared-memory carve-up, identical on host and device.
 struct TCSmem {
-  uint32_t k_off, p_off, alpha_off, bar_off, slot_off, plan_off, total;
+  uint32_t k_off, p_off, alpha_off, q_off, bar_off, slot_off, plan_off, total;
 };
-__host__ __device__ inline TCSmem tc_smem_layout(int CL, int TT, int d, int npad, int stages, int B) {
+__host__ __device__ inline TCSmem tc_smem_layout(int CL, int TT, int d, int stages, int B) {
   TCSmem s;
   const uint32_t dS = static_cast<uint32_t>(d / CL);
   uint32_t o = 0;
   s.k_off = o;
   o += static_cast<uint32_t>(stages) * TT * dS * 2u;
   s.p_off = o;
-  o += static_cast<uint32_t>(stages) * npad * TT * 2u;
+  o += static_cast<uint32_t>(stages) * kPRows * TT * 2u;
   s.alpha_off = o;
-  o += static_cast<uint32_t>(stages) * npad * 4u;
+  o += static_cast<uint32_t>(stages) * kPRows * 4u;
+  o = (o + 15u) & ~15u;
+  s.q_off = o;
+  o += dS * 4u;
   o = (o + 7u) & ~7u;
   s.bar_off = o;
-  o += (5u * stages + 1u) * 8u;
+  o += (5u * stages + 2u) * 8u;
   s.slot_off = o;
   o += 16u;
   s.plan_off = o;
@@ -77,331 +95,411 @@ __host__ __device__ inline TCSmem tc_smem_layout(int CL, int TT, int d, int npad
   return s;
 }
 
+// Row of head n in the P operand / accumulator: heads n, n+4, ... share the
+// TMEM lane quarter n % 4, so the correction warps split the rows evenly.
+__host__ __device__ inline int p_row(int n) { return 16 * (n & 3) + (n >> 2); }
+
 template <int CL, int TT, int DHB, int HPW>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kTCThreads, 1)
     decode_b_tc_kernel(const __grid_constant__ CUtensorMap kmap, const DecodeTCParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int DH = DHB * 64;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = (CL > 1) ? cluster_ctarank() : 0u;
-  const uint32_t peer = rank ^ 1u;
-  const int slot = blockIdx.x / CL;
+  const int group = blockIdx.x / CL;
   const int dS = p.d / CL, col0 = static_cast<int>(rank) * dS;
-  const int ncb = dS / 64, ndt = dS / 128;
+  const int ncb = dS / 64;
   const int H_own = p.H / CL, head0 = static_cast<int>(rank) * H_own;
-  const int stages = p.stages, npad = p.npad;
-  const TCSmem L = tc_smem_layout(CL, TT, p.d, npad, stages, p.B);
+  const int stages = p.stages;
+  const TCSmem L = tc_smem_layout(CL, TT, p.d, stages, p.B);
   uint8_t* kst = smem + L.k_off;
   uint8_t* pst = smem + L.p_off;
   float* alpha_s = reinterpret_cast<float*>(smem + L.alpha_off);
+  float* q_s = reinterpret_cast<float*>(smem + L.q_off);  // this CTA's columns of q
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar_off);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + stages;
-  uint64_t* pfull = bars + 2 * stages;
-  uint64_t* pempty = bars + 3 * stages;
-  uint64_t* corr = bars + 4 * stages;
-  uint64_t* accfull = bars + 5 * stages;
+  uint64_t* full = bars;                       // TMA landed (tx bytes)
+  uint64_t* empty = bars + stages;             // this CTA's MMAs done with the K stage
+  uint64_t* pfull = bars + 2 * stages;         // P and alpha of every softmax warp of the cluster written
+  uint64_t* pempty = bars + 3 * stages;        // every CTA's MMAs done with the P stage
+  uint64_t* corr = bars + 4 * stages;          // accumulator corrected for this tile's new maxima
+  uint64_t* accfull = bars + 5 * stages;       // last MMA of an item completed
+  uint64_t* accempty = bars + 5 * stages + 1;  // epilogue finished reading the accumulator
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.slot_off);
   int* s_nb = reinterpret_cast<int*>(smem + L.plan_off);
   int* s_rows = s_nb + (p.B + 1);
   int* s_off = s_rows + (p.B + 1);
   const uint32_t kstage_bytes = static_cast<uint32_t>(TT) * dS * 2u;
-  const uint32_t pstage_bytes = static_cast<uint32_t>(npad) * TT * 2u;
-
-  pdl_launch_dependents();
+  const uint32_t pstage_bytes = static_cast<uint32_t>(kPRows) * TT * 2u;
+  // K stage layout: [TT/16 slabs][ncb column blocks][16 rows][128 bytes], 128-byte swizzled
+  const uint32_t slab_bytes = static_cast<uint32_t>(ncb) * 2048u;
 
   // ---------------------------------------------------------------- set-up
+  // Nothing before pdl_wait_primary() reads memory that earlier work in the
+  // stream may still be writing (lengths, caches, queries, workspace).
   if (warp == 0) {
-    plan_split(p.lens, p.B, p.cap, p.append, p.n_slots, p.min_rows, s_nb, s_rows, s_off, p.ws_meta, p.status,
-               blockIdx.x == 0);
     if (lane == 0) tma_prefetch_desc(&kmap);
   } else if (warp == 1) {
     if (lane == 0) {
       for (int s = 0; s < stages; ++s) {
         mbar_init(&full[s], 1);
         mbar_init(&empty[s], 1);
-        mbar_init(&pfull[s], 4 * CL);
+        mbar_init(&pfull[s], kSoftmaxWarps * CL);
         mbar_init(&pempty[s], CL);
         mbar_init(&corr[s], 4);
       }
       mbar_init(accfull, 1);
+      mbar_init(accempty, 4);
       fence_barrier_init();
     }
     __syncwarp();
     tmem_alloc(tmem_slot, p.tmem_cols);
     tmem_relinquish();
-  } else {
-    // P buffers start at zero (padded heads stay zero); every alpha starts at 1.
-    const int t = threadIdx.x - 64;
+  } else if (warp >= 6) {
+    // P buffers start at zero (rows of absent heads stay zero); every alpha starts at 1.
+    const int t = threadIdx.x - 6 * 32;
     uint32_t* pz = reinterpret_cast<uint32_t*>(pst);
-    for (uint32_t i = t; i < stages * pstage_bytes / 4u; i += 128) pz[i] = 0u;
-    for (int i = t; i < stages * npad; i += 128) alpha_s[i] = 1.0f;
+    for (uint32_t i = t; i < stages * pstage_bytes / 4u; i += kSoftmaxWarps * 32) pz[i] = 0u;
+    for (int i = t; i < stages * kPRows; i += kSoftmaxWarps * 32) alpha_s[i] = 1.0f;
     fence_proxy_async_smem();
   }
+  pdl_wait_primary();
+  pdl_launch_dependents();
+  if (warp == 0)
+    plan_split(p.lens, p.B, p.cap, p.append, p.n_groups, p.max_items, p.min_rows, s_nb, s_rows, s_off, p.ws_meta,
+               p.status, blockIdx.x == 0);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (CL > 1) cluster_sync();
   const uint32_t tmem = *tmem_slot;
-
-  const SplitItem it = plan_lookup(slot, p.B, s_nb, s_rows, s_off);
-  const int ntiles = (it.b >= 0) ? (it.row1 - it.row0 + TT - 1) / TT : 0;
-  const int b = it.b;
-  bool failed = false;
+  const int n_items = s_off[p.B];
+  auto tiles_of = [&](const SplitItem& it) { return (it.row1 - it.row0 + TT - 1) / TT; };
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && ntiles > 0) {
+    if (lane == 0) {
       const uint64_t pol = l2_policy_evict_first();
-      int issued = 0;
-      for (int t = 0; t < ntiles; ++t) {
-        const int s = t % stages;
-        const uint32_t ph = static_cast<uint32_t>(t / stages) & 1u;
-        if (t >= stages && !mbar_wait(&empty[s], ph ^ 1u, p.status)) {
-          failed = true;
-          break;
-        }
-        const int r_lo = it.row0 + t * TT;
-        const int nbox = (min(TT, it.row1 - r_lo) + 15) / 16;
-        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nbox) * 16u * 128u * ncb);
-        const int y0 = static_cast<int>(static_cast<int64_t>(b) * p.cap + r_lo);
-        uint8_t* dst = kst + s * kstage_bytes;
-        for (int cb = 0; cb < ncb; ++cb)
+      int g = 0;  // tiles issued so far (all items)
+      bool ok = true;
+      for (int item = group; item < n_items && ok; item += p.n_groups) {
+        const SplitItem it = plan_lookup(item, p.B, s_nb, s_rows, s_off);
+        const int nt = tiles_of(it);
+        for (int t = 0; t < nt; ++t, ++g) {
+          const int s = g % stages;
+          const uint32_t ph = static_cast<uint32_t>(g / stages) & 1u;
+          if (g >= stages && !mbar_wait(&empty[s], ph ^ 1u, p.status)) {
+            ok = false;
+            break;
+          }
+          const int r_lo = it.row0 + t * TT;
+          const int nbox = (min(TT, it.row1 - r_lo) + 15) / 16;
+          mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(nbox) * slab_bytes);
+          const int y0 = static_cast<int>(static_cast<int64_t>(it.b) * p.cap + r_lo);
+          uint8_t* dst = kst + s * kstage_bytes;
+          // one 3-D box per 16-row slab: 64 columns x 16 rows x every column block of this CTA
           for (int rb = 0; rb < nbox; ++rb)
-            tma_load_2d(dst + cb * TT * 128 + rb * 16 * 128, &kmap, col0 + cb * 64, y0 + rb * 16, &full[s], pol);
-        issued = t + 1;
+            tma_load_3d(dst + rb * slab_bytes, &kmap, 0, y0 + rb * 16, col0 / 64, &full[s], pol);
+        }
       }
       // drain: every issued copy must land before the CTA can exit
-      for (int t = max(0, issued - stages); t < issued; ++t)
+      for (int t = max(0, g - stages); t < g; ++t)
         mbar_wait(&full[t % stages], static_cast<uint32_t>(t / stages) & 1u, p.status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && ntiles > 0) {
-      const uint32_t idesc = idesc_bf16_f32(128, static_cast<uint32_t>(npad), 1u, 0u);
+    if (lane == 0) {
       const uint32_t kbase = smem_u32(kst), pbase = smem_u32(pst);
-      for (int t = 0; t < ntiles; ++t) {
-        const int s = t % stages;
-        const uint32_t ph = static_cast<uint32_t>(t / stages) & 1u;
-        if (!mbar_wait(&corr[s], ph, p.status) || !mbar_wait(&full[s], ph, p.status)) {
-          failed = true;
-          break;
-        }
-        tc_fence_after();
-        const int r_lo = it.row0 + t * TT;
-        const int nks = (min(TT, it.row1 - r_lo) + 15) / 16;
-        const uint32_t ka = kbase + s * kstage_bytes, pa = pbase + s * pstage_bytes;
-        for (int j = 0; j < ndt; ++j) {
-          for (int kk = 0; kk < nks; ++kk) {
-            const uint64_t ad = smem_desc(ka + (2 * j) * TT * 128 + kk * 16 * 128, TT * 128, 1024, kLayoutSW128);
-            const uint64_t bd = smem_desc(pa + kk * 2 * 128, 128, (TT / 8) * 128, kLayoutNone);
-            umma_f16(tmem + static_cast<uint32_t>(j * npad), ad, bd, idesc, (t > 0 || kk > 0) ? 1u : 0u);
+      int g = 0, ii = 0;
+      bool ok = true;
+      for (int item = group; item < n_items && ok; item += p.n_groups, ++ii) {
+        const SplitItem it = plan_lookup(item, p.B, s_nb, s_rows, s_off);
+        const int nt = tiles_of(it);
+        // the previous item's epilogue must have read the accumulator
+        if (ii > 0 && !mbar_wait(accempty, static_cast<uint32_t>(ii - 1) & 1u, p.status)) break;
+        for (int t = 0; t < nt; ++t, ++g) {
+          const int s = g % stages;
+          const uint32_t ph = static_cast<uint32_t>(g / stages) & 1u;
+          if (!mbar_wait(&corr[s], ph, p.status) || !mbar_wait(&full[s], ph, p.status)) {
+            ok = false;
+            break;
           }
-        }
-        umma_commit(&empty[s]);
-        if (CL > 1) umma_commit_mc(&pempty[s], static_cast<uint16_t>((1u << CL) - 1u));
-        else umma_commit(&pempty[s]);
-      }
-      umma_commit(accfull);
-      mbar_wait(accfull, 0, p.status);  // no MMA may be in flight at teardown
-    }
-  } else if (ntiles > 0) {
-    // ------------------------------------------------------------ softmax warps
-    const int sw = warp - 2;        // 0..3
-    const int quarter = warp & 3;   // TMEM lane quarter this warp may access
-    const int rr = lane >> 3, jj = lane & 7;
-    float qr[HPW][DHB][8];
-    float mref[HPW], lsum[HPW];
-#pragma unroll
-    for (int k = 0; k < HPW; ++k) {
-      mref[k] = -INFINITY;
-      lsum[k] = 0.f;
-      const int hh = sw + 4 * k;
-#pragma unroll
-      for (int c = 0; c < DHB; ++c) {
-        if (hh < H_own) {
-          const float4* src =
-              reinterpret_cast<const float4*>(p.q + static_cast<size_t>(b) * p.d + col0 + hh * DH + c * 64 + jj * 8);
-          const float4 a0 = __ldg(src), a1 = __ldg(src + 1);
-          qr[k][c][0] = a0.x; qr[k][c][1] = a0.y; qr[k][c][2] = a0.z; qr[k][c][3] = a0.w;
-          qr[k][c][4] = a1.x; qr[k][c][5] = a1.y; qr[k][c][6] = a1.z; qr[k][c][7] = a1.w;
-        } else {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) qr[k][c][e] = 0.f;
-        }
-      }
-    }
-    const int nb_old = it.nb - p.append;  // rows holding cached keys
-    const uint32_t pst_base = smem_u32(pst);
-    const uint32_t alpha_base = smem_u32(alpha_s);
-
-    for (int t = 0; t < ntiles; ++t) {
-      const int s = t % stages;
-      const uint32_t ph = static_cast<uint32_t>(t / stages) & 1u;
-      const int r_lo = it.row0 + t * TT;
-      const int nvalid = min(TT, it.row1 - r_lo);
-      const int nloaded = (nvalid + 15) & ~15;
-      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph, p.status))) { failed = true; break; }
-      uint8_t* ks = kst + s * kstage_bytes;
-
-      // Rows >= nb_old in this tile hold no cached key: the appended key goes
-      // to row nb_old (also written to the cache), the rest become zero. Each
-      // warp fixes the column blocks of its own heads, which are the only
-      // columns it reads before the MMA (ordered by the proxy fence below).
-      if (r_lo + nloaded > nb_old) {
-        const int fr0 = max(nb_old - r_lo, 0);
-#pragma unroll
-        for (int k = 0; k < HPW; ++k) {
-          const int hh = sw + 4 * k;
-          if (hh >= H_own) continue;
-#pragma unroll
-          for (int c = 0; c < DHB; ++c) {
-            const int cb = hh * DHB + c;
-            for (int i = lane; i < (nloaded - fr0) * 8; i += 32) {
-              const int row = fr0 + (i >> 3), j = i & 7;
-              uint4 v = make_uint4(0u, 0u, 0u, 0u);
-              if (p.append && r_lo + row == nb_old) {
-                const size_t col = static_cast<size_t>(col0) + cb * 64 + j * 8;
-                v = __ldg(reinterpret_cast<const uint4*>(p.k_new + static_cast<size_t>(b) * p.d + col));
-                *reinterpret_cast<uint4*>(p.kcache + (static_cast<size_t>(b) * p.cap + nb_old) * p.d + col) = v;
-              }
-              *reinterpret_cast<uint4*>(ks + cb * TT * 128 + row * 128 + ((j ^ (row & 7)) << 4)) = v;
+          tc_fence_after();
+          const int r_lo = it.row0 + t * TT;
+          const int nks = (min(TT, it.row1 - r_lo) + 15) / 16;
+          const uint32_t ka = kbase + s * kstage_bytes, pa = pbase + s * pstage_bytes;
+          for (int kk = 0; kk < nks; ++kk) {
+            const uint64_t ad = smem_desc(pa + kk * 256, 128, (TT / 8) * 128, kLayoutNone);
+            for (int c = 0; c < dS; c += 256) {
+              const int hf = c >> 9, n0 = c & 511;
+              const int N = min(256, dS - c);
+              const uint64_t bd = smem_desc(ka + kk * slab_bytes + (c / 64) * 2048, 2048, 1024, kLayoutSW128);
+              umma_f16(tmem + (static_cast<uint32_t>(16 * hf) << 16) + static_cast<uint32_t>(n0), ad, bd,
+                       idesc_bf16_f32(kPRows, static_cast<uint32_t>(N), 0u, 1u), (t > 0 || kk > 0) ? 1u : 0u);
             }
           }
+          umma_commit(&empty[s]);
+          if (CL > 1) umma_commit_mc(&pempty[s], static_cast<uint16_t>((1u << CL) - 1u));
+          else umma_commit(&pempty[s]);
         }
-        __syncwarp();
+        umma_commit(accfull);  // also after a failed tile: covers every MMA issued so far
+        if (!ok) {
+          ++ii;
+          break;
+        }
       }
-
-      // P stage s is free once the MMAs that read it (tile t - stages) finished in every CTA.
-      if (t >= stages && !__all_sync(0xffffffffu, mbar_wait(&pempty[s], ph ^ 1u, p.status))) {
-        failed = true;
-        break;
-      }
-
-      float alpha_k[HPW];
-#pragma unroll
-      for (int k = 0; k < HPW; ++k) {
-        const int hh = sw + 4 * k;
-        alpha_k[k] = 1.f;
-        if (hh >= H_own) continue;
-        float sv[TT / 4];
-#pragma unroll
-        for (int g = 0; g < TT / 4; ++g) {
-          const int row = 4 * g + rr;
-          float acc = 0.f;
-#pragma unroll
-          for (int c = 0; c < DHB; ++c) {
-            const int cb = (hh * DH) / 64 + c;
-            const uint4 v = *reinterpret_cast<const uint4*>(ks + cb * TT * 128 + row * 128 + ((jj ^ (row & 7)) << 4));
-            acc = fmaf(qr[k][c][0], bf16lo(v.x), acc);
-            acc = fmaf(qr[k][c][1], bf16hi(v.x), acc);
-            acc = fmaf(qr[k][c][2], bf16lo(v.y), acc);
-            acc = fmaf(qr[k][c][3], bf16hi(v.y), acc);
-            acc = fmaf(qr[k][c][4], bf16lo(v.z), acc);
-            acc = fmaf(qr[k][c][5], bf16hi(v.z), acc);
-            acc = fmaf(qr[k][c][6], bf16lo(v.w), acc);
-            acc = fmaf(qr[k][c][7], bf16hi(v.w), acc);
+      // no MMA may be in flight at teardown: wait for the last commit
+      if (ii > 0) mbar_wait(accfull, static_cast<uint32_t>(ii - 1) & 1u, p.status);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ correction + epilogue warpgroup
+    // Lane l of quarter q holds head n = 4*(l % 16) + q in accumulator half l / 16.
+    const int quarter = warp & 3;
+    const int n = 4 * (lane & 15) + quarter, hf = lane >> 4;
+    const int hcols = min(512, dS);  // columns per accumulator half
+    const int my_cols = min(512, max(dS - 512 * hf, 0));
+    const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    int g = 0, ii = 0;
+    bool ok = true;
+    for (int item = group; item < n_items && ok; item += p.n_groups, ++ii) {
+      const SplitItem it = plan_lookup(item, p.B, s_nb, s_rows, s_off);
+      const int nt = tiles_of(it);
+      for (int t = 0; t < nt; ++t, ++g) {
+        const int s = g % stages;
+        const uint32_t ph = static_cast<uint32_t>(g / stages) & 1u;
+        if (!__all_sync(0xffffffffu, mbar_wait(&pfull[s], ph, p.status))) {
+          ok = false;
+          break;
+        }
+        const float alpha = (n < p.H) ? alpha_s[s * kPRows + n] : 1.f;
+        if (t > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+          // rescale this quarter's rows once the previous tile's MMAs have finished
+          const int sp = (g - 1) % stages;
+          const uint32_t php = static_cast<uint32_t>((g - 1) / stages) & 1u;
+          if (!__all_sync(0xffffffffu, mbar_wait(&empty[sp], php, p.status))) {
+            ok = false;
+            break;
           }
-          acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-          acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-          acc += __shfl_xor_sync(0xffffffffu, acc, 4);
-          sv[g] = (row < nvalid) ? acc * p.scale_log2 : -INFINITY;
-        }
-        float mx = sv[0];
-#pragma unroll
-        for (int g = 1; g < TT / 4; ++g) mx = fmaxf(mx, sv[g]);
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-        if (t == 0) {
-          mref[k] = mx;
-        } else if (mx > mref[k] + 8.f) {
-          alpha_k[k] = exp2f(mref[k] - mx);
-          mref[k] = mx;
-          lsum[k] *= alpha_k[k];
-        }
-        // lane (rr, jj) owns row 4*jj + rr of the tile
-        float sel = sv[0];
-#pragma unroll
-        for (int g = 1; g < TT / 4; ++g) sel = (jj == g) ? sv[g] : sel;
-        const int trow = 4 * jj + rr;
-        if (jj < TT / 4) {
-          const float pv = (trow < nvalid) ? exp2f(sel - mref[k]) : 0.f;
-          const __nv_bfloat16 pb = __float2bfloat16_rn(pv);
-          lsum[k] += __bfloat162float(pb);
-          const int n = head0 + hh;
-          const uint32_t off = static_cast<uint32_t>(s) * pstage_bytes +
-                               static_cast<uint32_t>(((n >> 3) * (TT / 8) + (trow >> 3)) * 128 + (n & 7) * 16 +
-                                                     (trow & 7) * 2);
-          const uint16_t bits = __bfloat16_as_ushort(pb);
-          asm volatile("st.shared.u16 [%0], %1;" ::"r"(pst_base + off), "h"(bits) : "memory");
-          if (CL > 1) st_cluster_u16(mapa_shared(pst_base + off, peer), bits);
-        }
-        if (lane == 0) {
-          const uint32_t aoff = static_cast<uint32_t>((s * npad + head0 + hh) * 4);
-          alpha_s[s * npad + head0 + hh] = alpha_k[k];
-          if (CL > 1) st_cluster_f32(mapa_shared(alpha_base + aoff, peer), alpha_k[k]);
-        }
-      }
-      fence_proxy_async_smem();
-      if (CL > 1) fence_proxy_async_cluster();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&pfull[s]);
-        if (CL > 1) mbar_arrive_cluster(mapa_shared(smem_u32(&pfull[s]), peer));
-      }
-
-      // Lazy rescale: every CTA multiplies its TMEM columns of head n by the
-      // alpha published for n, after the MMAs of the previous tile finished.
-      if (!__all_sync(0xffffffffu, mbar_wait(&pfull[s], ph, p.status))) { failed = true; break; }
-      const float my_alpha = (lane < npad) ? alpha_s[s * npad + lane] : 1.f;
-      if (t > 0 && __any_sync(0xffffffffu, my_alpha != 1.f)) {
-        const int sp = (t - 1) % stages;
-        const uint32_t php = static_cast<uint32_t>((t - 1) / stages) & 1u;
-        if (!__all_sync(0xffffffffu, mbar_wait(&empty[sp], php, p.status))) { failed = true; break; }
-        tc_fence_after();
-        for (int j = 0; j < ndt; ++j) {
-          for (int c16 = 0; c16 < npad; c16 += 16) {
-            const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + j * npad + c16;
+          tc_fence_after();
+          for (int c = 0; c < hcols; c += 16) {
             float v[16];
-            tmem_ld16(ta, v);
+            tmem_ld16(tbase + c, v);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] *= __shfl_sync(0xffffffffu, my_alpha, (c16 + i) & 31);
-            tmem_st16(ta, v);
+            for (int i = 0; i < 16; ++i) v[i] *= alpha;
+            tmem_st16(tbase + c, v);
           }
+          tmem_wait_st();
         }
-        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&corr[s]);
+      }
+      if (!ok) break;
+      // epilogue: accumulator rows -> partial U[item][head][own columns]
+      if (!__all_sync(0xffffffffu, mbar_wait(accfull, static_cast<uint32_t>(ii) & 1u, p.status))) break;
+      tc_fence_after();
+      float* dst = p.ws_U + (static_cast<size_t>(item) * p.H + n) * p.d + col0 + 512 * hf;
+      for (int c = 0; c < hcols; c += 16) {
+        float v[16];
+        tmem_ld16(tbase + c, v);
+        tmem_wait_ld();
+        if (n < p.H && c < my_cols) {
+#pragma unroll
+          for (int i = 0; i < 16; i += 4)
+            *reinterpret_cast<float4*>(dst + c + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+        }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&corr[s]);
+      if (lane == 0) mbar_arrive(accempty);
     }
-
-    // ------------------------------------------------------------ epilogue
-    if (!failed && __all_sync(0xffffffffu, mbar_wait(accfull, 0, p.status))) {
-      tc_fence_after();
-      const size_t item = static_cast<size_t>(slot);
-      for (int j = 0; j < ndt; ++j) {
-        for (int c16 = 0; c16 < npad; c16 += 16) {
-          float v[16];
-          tmem_ld16(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + j * npad + c16, v);
-          tmem_wait_ld();
-          const int dcol = col0 + j * 128 + quarter * 32 + lane;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int n = c16 + i;
-            if (n < p.H) p.ws_U[(item * p.H + n) * p.d + dcol] = v[i];
-          }
-        }
-      }
+  } else {
+    // ------------------------------------------------------------ score / softmax warps
+    const int sw = warp - 6;  // heads sw, sw + 8, ... of this CTA
+    const int gq = lane >> 2, tq = lane & 3;  // mma.sync fragment coordinates
+    const uint32_t kbase = smem_u32(kst);
+    const uint32_t pst_base = smem_u32(pst);
+    const uint32_t alpha_base = smem_u32(alpha_s);
+    int g = 0;
+    bool ok = true;
+    for (int item = group; item < n_items && ok; item += p.n_groups) {
+      const SplitItem it = plan_lookup(item, p.B, s_nb, s_rows, s_off);
+      const int nt = tiles_of(it);
+      const int b = it.b;
+      const int nb_old = it.nb - p.append;  // rows holding cached keys
+      // q of this warp's heads: to shared memory, then B fragments (column 0 = bf16 high part,
+      // column 1 = bf16 low part of q, other columns zero)
+      uint32_t bq[HPW][DHB * 4][2];
+      float mref[HPW], lsum[HPW];
+      __syncwarp();
 #pragma unroll
       for (int k = 0; k < HPW; ++k) {
-        const int hh = sw + 4 * k;
+        const int hh = sw + kSoftmaxWarps * k;
+        mref[k] = -INFINITY;
+        lsum[k] = 0.f;
+        if (hh < H_own) {
+          const float* src = p.q + static_cast<size_t>(b) * p.d + col0 + hh * DH;
+          for (int i = lane; i < DH / 4; i += 32)
+            reinterpret_cast<float4*>(q_s + hh * DH)[i] = __ldg(reinterpret_cast<const float4*>(src) + i);
+        }
+      }
+      __syncwarp();
+#pragma unroll
+      for (int k = 0; k < HPW; ++k) {
+        const int hh = sw + kSoftmaxWarps * k;
+#pragma unroll
+        for (int ks = 0; ks < DHB * 4; ++ks) {
+          uint32_t v0 = 0, v1 = 0;
+          if (hh < H_own && gq < 2) {
+            const float* qc = q_s + hh * DH + ks * 16 + 2 * tq;
+            const float x0 = qc[0], x1 = qc[1], x8 = qc[8], x9 = qc[9];
+            if (gq == 0) {
+              v0 = pack_bf16x2(x0, x1);
+              v1 = pack_bf16x2(x8, x9);
+            } else {
+              v0 = pack_bf16x2(x0 - __bfloat162float(__float2bfloat16_rn(x0)),
+                               x1 - __bfloat162float(__float2bfloat16_rn(x1)));
+              v1 = pack_bf16x2(x8 - __bfloat162float(__float2bfloat16_rn(x8)),
+                               x9 - __bfloat162float(__float2bfloat16_rn(x9)));
+            }
+          }
+          bq[k][ks][0] = v0;
+          bq[k][ks][1] = v1;
+        }
+      }
+
+      for (int t = 0; t < nt; ++t, ++g) {
+        const int s = g % stages;
+        const uint32_t ph = static_cast<uint32_t>(g / stages) & 1u;
+        const int r_lo = it.row0 + t * TT;
+        const int nvalid = min(TT, it.row1 - r_lo);
+        const int nloaded = (nvalid + 15) & ~15;
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph, p.status))) {
+          ok = false;
+          break;
+        }
+        uint8_t* ks_ptr = kst + s * kstage_bytes;
+
+        // Rows >= nb_old in this tile hold no cached key: the appended key goes
+        // to row nb_old (also written to the cache), the rest become zero. Each
+        // warp fixes the column blocks of its own heads; the MMA reads them
+        // after the proxy fence and the pfull/corr barriers below.
+        if (r_lo + nloaded > nb_old) {
+          const int fr0 = max(nb_old - r_lo, 0);
+#pragma unroll
+          for (int k = 0; k < HPW; ++k) {
+            const int hh = sw + kSoftmaxWarps * k;
+            if (hh >= H_own) continue;
+#pragma unroll
+            for (int c = 0; c < DHB; ++c) {
+              const int cb = hh * DHB + c;
+              for (int i = lane; i < (nloaded - fr0) * 8; i += 32) {
+                const int rw = fr0 + (i >> 3), j = i & 7;
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (p.append && r_lo + rw == nb_old) {
+                  const size_t col = static_cast<size_t>(col0) + cb * 64 + j * 8;
+                  v = __ldg(reinterpret_cast<const uint4*>(p.k_new + static_cast<size_t>(b) * p.d + col));
+                  *reinterpret_cast<uint4*>(p.kcache + (static_cast<size_t>(b) * p.cap + nb_old) * p.d + col) = v;
+                }
+                *reinterpret_cast<uint4*>(ks_ptr + (rw >> 4) * slab_bytes + cb * 2048 + (rw & 15) * 128 +
+                                          ((j ^ (rw & 7)) << 4)) = v;
+              }
+            }
+          }
+          __syncwarp();
+        }
+
+        // P stage s is free once the MMAs that read it (tile g - stages) finished in every CTA.
+        if (g >= stages && !__all_sync(0xffffffffu, mbar_wait(&pempty[s], ph ^ 1u, p.status))) {
+          ok = false;
+          break;
+        }
+
+        const uint32_t kt = kbase + s * kstage_bytes;
+#pragma unroll
+        for (int k = 0; k < HPW; ++k) {
+          const int hh = sw + kSoftmaxWarps * k;
+          if (hh >= H_own) continue;
+          // scores of rows (16 rb + gq) and (16 rb + gq + 8) in lanes with tq == 0
+          float sc[TT / 8];
+#pragma unroll
+          for (int rb = 0; rb < TT / 16; ++rb) {
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            // ldmatrix.x4: lanes 0-7 rows 0-7 / k 0-7, 8-15 rows 8-15 / k 0-7,
+            // 16-23 rows 0-7 / k 8-15, 24-31 rows 8-15 / k 8-15 of the 16x16 A tile
+            const int row = rb * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
+#pragma unroll
+            for (int ks = 0; ks < DHB * 4; ++ks) {
+              const int colk = hh * DH + ks * 16 + (lane >> 4) * 8;  // first column of this lane's 8x8 matrix
+              const uint32_t addr = kt + (row >> 4) * slab_bytes + (colk >> 6) * 2048 + (row & 15) * 128 +
+                                    ((((colk & 63) >> 3) ^ (row & 7)) << 4);
+              uint32_t a[4];
+              ldmatrix_x4(addr, a);
+              mma_16816_bf16(acc, a, bq[k][ks][0], bq[k][ks][1]);
+            }
+            sc[2 * rb] = acc[0] + acc[1];
+            sc[2 * rb + 1] = acc[2] + acc[3];
+          }
+          float mx = -INFINITY;
+#pragma unroll
+          for (int i = 0; i < TT / 8; ++i) {
+            const int trow = 8 * i + gq;  // (rb, half) = (i / 2, i % 2): row 16 rb + 8 half + gq
+            sc[i] = (tq == 0 && trow < nvalid) ? sc[i] * p.scale_log2 : -INFINITY;
+            mx = fmaxf(mx, sc[i]);
+          }
+          mx = warp_max(mx);
+          float alpha = 1.f;
+          if (t == 0) {
+            mref[k] = mx;
+          } else if (mx > mref[k] + kLazyRescaleLog2) {
+            alpha = exp2f(mref[k] - mx);
+            mref[k] = mx;
+            lsum[k] *= alpha;
+          }
+          const int n = head0 + hh;
+          const int m = p_row(n);
+          if (tq == 0) {
+#pragma unroll
+            for (int i = 0; i < TT / 8; ++i) {
+              const int trow = 8 * i + gq;
+              const float pv = (trow < nvalid) ? exp2f(sc[i] - mref[k]) : 0.f;
+              const __nv_bfloat16 pb = __float2bfloat16_rn(pv);
+              lsum[k] += __bfloat162float(pb);
+              const uint32_t off = static_cast<uint32_t>(s) * pstage_bytes +
+                                   static_cast<uint32_t>(((m >> 3) * (TT / 8) + i) * 128 + (m & 7) * 16 + gq * 2);
+              const uint16_t bits = __bfloat16_as_ushort(pb);
+              asm volatile("st.shared.u16 [%0], %1;" ::"r"(pst_base + off), "h"(bits) : "memory");
+#pragma unroll
+              for (int r = 1; r < CL; ++r) st_cluster_u16(mapa_shared(pst_base + off, (rank + r) % CL), bits);
+            }
+          }
+          if (lane == 0) {
+            alpha_s[s * kPRows + n] = alpha;
+#pragma unroll
+            for (int r = 1; r < CL; ++r)
+              st_cluster_f32(mapa_shared(alpha_base + static_cast<uint32_t>((s * kPRows + n) * 4), (rank + r) % CL),
+                             alpha);
+          }
+        }
+        fence_proxy_async_smem();
+        if (CL > 1) fence_proxy_async_cluster();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(&pfull[s]);
+#pragma unroll
+          for (int r = 1; r < CL; ++r) mbar_arrive_cluster(mapa_shared(smem_u32(&pfull[s]), (rank + r) % CL));
+        }
+      }
+      if (!ok) break;
+      const size_t slot = static_cast<size_t>(item);
+#pragma unroll
+      for (int k = 0; k < HPW; ++k) {
+        const int hh = sw + kSoftmaxWarps * k;
         const float tot = warp_sum(lsum[k]);
         if (hh < H_own && lane == 0) {
-          p.ws_m[item * p.H + head0 + hh] = mref[k];
-          p.ws_l[item * p.H + head0 + hh] = tot;
+          p.ws_m[slot * p.H + head0 + hh] = mref[k];
+          p.ws_l[slot * p.H + head0 + hh] = tot;
         }
       }
     }
@@ -421,9 +519,25 @@ __global__ void __launch_bounds__(192, 1)
 namespace {
 
 struct TCConfig {
-  int CL, TT, DHB, HPW, stages, npad;
+  int CL, TT, DHB, HPW, stages;
   uint32_t tmem_cols, smem;
 };
+
+// Template instances compiled below (CL, TT, DHB, HPW); pick_config only returns these.
+#define SLIM_TC_INSTANCES(X)                                                                               \
+  X(1, 32, 1, 1) X(1, 32, 1, 2) X(1, 32, 1, 3) X(1, 32, 1, 4) X(1, 32, 2, 1) X(1, 32, 2, 2) X(2, 32, 1, 1) \
+  X(2, 32, 1, 2) X(2, 32, 1, 3) X(2, 32, 1, 4) X(2, 32, 2, 1) X(2, 32, 2, 2) X(4, 32, 1, 1) X(4, 32, 1, 2) \
+  X(4, 32, 2, 1) X(4, 32, 2, 2) X(1, 16, 1, 1) X(1, 16, 1, 2) X(1, 16, 1, 3) X(1, 16, 1, 4) X(1, 16, 2, 1) \
+  X(1, 16, 2, 2) X(2, 16, 1, 1) X(2, 16, 1, 2) X(2, 16, 1, 3) X(2, 16, 1, 4) X(2, 16, 2, 1) X(2, 16, 2, 2) \
+  X(4, 16, 1, 1) X(4, 16, 1, 2) X(4, 16, 2, 1) X(4, 16, 2, 2)
+
+bool tc_instantiated(int CL, int TT, int DHB, int HPW) {
+#define SLIM_TC_MATCH(a, b, c, e) \
+  if (CL == a && TT == b && DHB == c && HPW == e) return true;
+  SLIM_TC_INSTANCES(SLIM_TC_MATCH)
+#undef SLIM_TC_MATCH
+  return false;
+}
 
 uint32_t pow2_cols(uint32_t c) {
   uint32_t r = 32;
@@ -431,53 +545,32 @@ uint32_t pow2_cols(uint32_t c) {
   return r;
 }
 
-// Template instances compiled below (CL, TT, DHB, HPW); pick_config only returns these.
-#define SLIM_TC_INSTANCES(X)                                                                          \
-  X(1, 32, 1, 2) X(1, 32, 1, 4) X(1, 32, 1, 5) X(1, 32, 1, 8) X(1, 16, 1, 2) X(1, 16, 1, 4) X(1, 16, 1, 5) \
-  X(1, 16, 1, 8) X(1, 32, 2, 2) X(1, 32, 2, 4) X(1, 16, 2, 2) X(1, 16, 2, 4) X(2, 32, 1, 2) X(2, 32, 1, 4) \
-  X(2, 16, 1, 2) X(2, 16, 1, 4) X(2, 16, 1, 8) X(2, 32, 2, 2) X(2, 32, 2, 4) X(2, 16, 2, 2) X(2, 16, 2, 4)
-
-bool tc_instantiated(int CL, int TT, int DHB, int HPW) {
-#define SLIM_TC_MATCH(a, b, c, e) if (CL == a && TT == b && DHB == c && HPW == e) return true;
-  SLIM_TC_INSTANCES(SLIM_TC_MATCH)
-#undef SLIM_TC_MATCH
-  return false;
-}
-
 bool pick_config(int B, int d, int H, TCConfig* out) {
-  if (H <= 0 || d % H) return false;
+  if (H <= 0 || d % H || H > kPRows) return false;
   const int dh = d / H;
   if (dh != 64 && dh != 128) return false;
   const int smem_cap = max_smem_optin();
-  const int npad = ((H + 15) / 16) * 16;
-  for (int CL = 1; CL <= 2; ++CL) {
-    if (d % (128 * CL) || H % CL || (d / CL) % dh) continue;
+  for (int CL = 1; CL <= 4; CL *= 2) {
+    if (d % (64 * CL) || H % CL || (d / CL) % dh || d / CL > kMaxColsPerCTA) continue;
     const int H_own = H / CL;
-    const int hpw = (H_own + 3) / 4;
-    int HPW = hpw <= 2 ? 2 : hpw <= 4 ? 4 : hpw <= 5 ? 5 : hpw <= 8 ? 8 : 0;
-    if (!HPW) continue;
-    if (npad > 32) continue;
-    const uint32_t cols = static_cast<uint32_t>((d / CL / 128) * npad);
-    if (cols > 512) continue;
+    const int HPW = (H_own + kSoftmaxWarps - 1) / kSoftmaxWarps;
     for (int TT : {32, 16}) {
       int stages = 0;
       for (int s = 8; s >= 2; --s) {
-        if (tc_smem_layout(CL, TT, d, npad, s, B).total <= static_cast<uint32_t>(smem_cap)) {
+        if (tc_smem_layout(CL, TT, d, s, B).total <= static_cast<uint32_t>(smem_cap)) {
           stages = s;
           break;
         }
       }
-      if (stages == 0) continue;
-      if (TT == 32 && stages < 3) continue;  // prefer more stages of 16 rows
+      if (stages < (TT == 32 ? 3 : 2)) continue;
       if (!tc_instantiated(CL, TT, dh / 64, HPW)) continue;
       out->CL = CL;
       out->TT = TT;
       out->DHB = dh / 64;
       out->HPW = HPW;
       out->stages = stages;
-      out->npad = npad;
-      out->tmem_cols = pow2_cols(cols);
-      out->smem = tc_smem_layout(CL, TT, d, npad, stages, B).total;
+      out->tmem_cols = pow2_cols(static_cast<uint32_t>(std::min(d / CL, 512)));
+      out->smem = tc_smem_layout(CL, TT, d, stages, B).total;
       return true;
     }
   }
@@ -490,17 +583,19 @@ cudaError_t launch_tc(const CUtensorMap& map, const DecodeTCParams& prm, const T
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(c.smem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(prm.n_slots * CL), 1, 1);
-  cfg.blockDim = dim3(192, 1, 1);
+  cfg.gridDim = dim3(static_cast<unsigned>(prm.n_groups * CL), 1, 1);
+  cfg.blockDim = dim3(kTCThreads, 1, 1);
   cfg.dynamicSmemBytes = c.smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = CL;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = CL;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = CL > 1 ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kern, map, prm);
 }
 
@@ -511,12 +606,17 @@ bool decode_b_tc_supported(int B, int d, int H) {
   return pick_config(B, d, H, &c);
 }
 
+int decode_b_tc_cluster(int B, int d, int H) {
+  TCConfig c;
+  return pick_config(B, d, H, &c) ? c.CL : 0;
+}
+
 cudaError_t launch_decode_b_tc(const DecodeArgs& a, const SplitWorkspace& ws, cudaStream_t st, int* launches) {
   TCConfig c;
   if (a.dtype != SLIM_BF16 || !pick_config(a.B, a.d, a.H, &c)) return cudaErrorNotSupported;
   CUtensorMap map;
-  if (!encode_tmap_2d_bf16(&map, a.kcache, static_cast<uint64_t>(a.d), static_cast<uint64_t>(a.B) * a.cap,
-                           static_cast<uint64_t>(a.d) * 2u, 64, 16, true))
+  // K cache viewed as [d/64 column blocks][B*cap rows][64 columns]; a box is 64 x 16 x (d/CL/64)
+  if (!encode_tmap_kslab(&map, a.kcache, static_cast<uint64_t>(a.B) * a.cap, a.d, a.d / c.CL / 64))
     return cudaErrorInvalidValue;
   DecodeTCParams prm;
   prm.q = a.q;
@@ -533,20 +633,18 @@ cudaError_t launch_decode_b_tc(const DecodeArgs& a, const SplitWorkspace& ws, cu
   prm.H = a.H;
   prm.cap = a.cap;
   prm.append = a.k_new != nullptr ? 1 : 0;
-  prm.n_slots = max(num_sms() / c.CL, a.B);
-  if (prm.n_slots > ws.max_items) return cudaErrorInvalidValue;
+  prm.n_groups = num_sms() / c.CL;
+  prm.max_items = ws.max_items;
   prm.stages = c.stages;
-  prm.npad = c.npad;
   prm.min_rows = max(16, 8 * a.H);
   prm.tmem_cols = c.tmem_cols;
   prm.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(a.d / a.H));
   cudaError_t e = cudaErrorNotSupported;
-#define SLIM_TC_CASE(CL_, TT_, DHB_, HPW_)                                                  \
-  if (c.CL == CL_ && c.TT == TT_ && c.DHB == DHB_ && c.HPW == HPW_) {                        \
-    e = launch_tc<CL_, TT_, DHB_, HPW_>(map, prm, c, st);                                    \
+#define SLIM_TC_CASE(CL_, TT_, DHB_, HPW_)                           \
+  if (c.CL == CL_ && c.TT == TT_ && c.DHB == DHB_ && c.HPW == HPW_) { \
+    e = launch_tc<CL_, TT_, DHB_, HPW_>(map, prm, c, st);             \
   } else
-  SLIM_TC_INSTANCES(SLIM_TC_CASE)
-  { e = cudaErrorNotSupported; }
+  SLIM_TC_INSTANCES(SLIM_TC_CASE) { e = cudaErrorNotSupported; }
 #undef SLIM_TC_CASE
   if (e == cudaSuccess && launches) ++*launches;
   return e;

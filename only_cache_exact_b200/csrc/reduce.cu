@@ -16,6 +16,8 @@
 // Ordering (a) needs only the merge (its partials are already softmax·V).
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "ptx.cuh"
 
 namespace slim {
@@ -28,56 +30,89 @@ struct ReduceBParams {
   const void* w_kv;
   float* out;
   int32_t* lens;
-  int B, d, H, ndb, bb, max_items;
+  int32_t* status;
+  int B, d, H, ndb, max_items;
+  int sb;           // sequences per cluster reduction round
 };
 
+constexpr int kReduceThreads = 256;
+constexpr int kReduceNBB = 8;  // sequences per projection block (register accumulators)
+
 template <typename WT>
-__device__ __forceinline__ float ldw(const WT* w, size_t i);
+struct WVec;
 template <>
-__device__ __forceinline__ float ldw<float>(const float* w, size_t i) {
-  return __ldg(w + i);
-}
+struct WVec<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ __forceinline__ static void load(const __nv_bfloat16* p, float (&w)[8]) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+    w[0] = bf16lo(v.x); w[1] = bf16hi(v.x); w[2] = bf16lo(v.y); w[3] = bf16hi(v.y);
+    w[4] = bf16lo(v.z); w[5] = bf16hi(v.z); w[6] = bf16lo(v.w); w[7] = bf16hi(v.w);
+  }
+};
 template <>
-__device__ __forceinline__ float ldw<__nv_bfloat16>(const __nv_bfloat16* w, size_t i) {
-  return __bfloat162float(w[i]);
+struct WVec<float> {
+  static constexpr int N = 4;
+  __device__ __forceinline__ static void load(const float* p, float (&w)[4]) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(p));
+    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+  }
+};
+
+struct ReduceSmem {
+  uint32_t wts, ubar, part, red, total;
+};
+__host__ __device__ inline ReduceSmem reduce_smem_layout(int max_items, int DB, int d_h, int sb) {
+  ReduceSmem r;
+  uint32_t o = 0;
+  r.wts = o;
+  o += ((static_cast<uint32_t>(max_items) + 3u) & ~3u) * 4u;
+  r.ubar = o;
+  o += static_cast<uint32_t>(kReduceNBB) * DB * 4u;
+  r.part = o;
+  o += static_cast<uint32_t>(sb) * d_h * 4u;
+  r.red = o;
+  o += static_cast<uint32_t>(kReduceThreads / 32) * kReduceNBB * d_h * 4u;
+  r.total = o;
+  return r;
 }
 
 template <typename WT>
-__global__ void __launch_bounds__(256) reduce_b_kernel(const ReduceBParams p) {
-  extern __shared__ float rsm[];
+__global__ void __launch_bounds__(kReduceThreads) reduce_b_kernel(const ReduceBParams p) {
+  extern __shared__ __align__(16) uint8_t rsm[];
+  constexpr int VEC = WVec<WT>::N;
   const int h = blockIdx.x, r = blockIdx.y;
   const int d_h = p.d / p.H;
   const int DB = p.d / p.ndb, c0 = r * DB;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const WT* W = static_cast<const WT*>(p.w_kv);
+  const ReduceSmem L = reduce_smem_layout(p.max_items, DB, d_h, p.sb);
+  float* wts = reinterpret_cast<float*>(rsm + L.wts);
+  float* ubar = reinterpret_cast<float*>(rsm + L.ubar);
+  float* part = reinterpret_cast<float*>(rsm + L.part);
+  float* red = reinterpret_cast<float*>(rsm + L.red);
 
-  // Before the partials exist: pull this CTA's W_KV block into L2.
+  // Before the partials exist: pull this CTA's W_KV block (rows c0.., head-h columns) into L2.
   {
     const int row_bytes = d_h * static_cast<int>(sizeof(WT));
     const int lines = (row_bytes + 127) / 128;
-    for (int i = tid; i < DB * lines; i += blockDim.x) {
+    for (int i = tid; i < DB * lines; i += kReduceThreads) {
       const int row = i / lines, ln = i % lines;
       const char* a = reinterpret_cast<const char*>(W + static_cast<size_t>(c0 + row) * p.d + h * d_h) + ln * 128;
       asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
     }
   }
   pdl_wait_primary();
+  pdl_launch_dependents();
+  __syncthreads();
 
-  const int items = p.meta[0];
   const int32_t* off = p.meta + 1;
-  float* wts = rsm;                         // [max_items]
-  float* ubar = wts + p.max_items;          // [bb][DB]
-  float* part = ubar + p.bb * DB;           // [bb][d_h]
-  float* red = part + p.bb * d_h;           // [groups][bb][d_h]
-
   if (h == 0 && r == 0) {
-    for (int b = tid; b < p.B; b += blockDim.x)
+    for (int b = tid; b < p.B; b += kReduceThreads)
       if (p.meta[2 + p.B + b] & kSeqAppend) p.lens[b] += 1;
   }
 
-  // merge weights 2^(m_c - M) / L for every item of head h
-  const int warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
-  for (int b = warp; b < p.B; b += nw) {
+  // merge weights 2^(m_c - M) / L of every item c for head h
+  for (int b = warp; b < p.B; b += kReduceThreads / 32) {
     const int c_lo = off[b], c_hi = off[b + 1];
     float M = -INFINITY;
     for (int c = c_lo + lane; c < c_hi; c += 32) M = fmaxf(M, p.m[static_cast<size_t>(c) * p.H + h]);
@@ -89,54 +124,104 @@ __global__ void __launch_bounds__(256) reduce_b_kernel(const ReduceBParams p) {
     const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
     for (int c = c_lo + lane; c < c_hi; c += 32) wts[c] = exp2f(p.m[static_cast<size_t>(c) * p.H + h] - M) * inv;
   }
-  (void)items;
   __syncthreads();
 
-  const int groups = blockDim.x / d_h;  // d_h <= 256
-  const int j = tid % d_h, g = tid / d_h;
+  const int ncg = d_h / VEC;               // column groups of VEC columns
+  const int G = kReduceThreads / ncg;      // row groups
+  const int cg = tid % ncg, g = tid / ncg;
+  const int gpw = 32 / ncg;                // row groups per warp (ncg <= 32)
   const uint32_t part_base = smem_u32(part);
 
-  for (int b0 = 0; b0 < p.B; b0 += p.bb) {
-    const int nbb = min(p.bb, p.B - b0);
-    // ū for the d-block of this CTA
-    for (int i = tid; i < nbb * DB; i += blockDim.x) {
-      const int bl = i / DB, col = i % DB;
-      const int b = b0 + bl;
-      float acc = 0.f;
-      for (int c = off[b]; c < off[b + 1]; ++c)
-        acc = fmaf(wts[c], p.U[(static_cast<size_t>(c) * p.H + h) * p.d + c0 + col], acc);
-      ubar[bl * DB + col] = acc;
-    }
-    __syncthreads();
-    // partial head output: ū[bl, block] · W_KV[block, h-cols]
-    if (g < groups) {
-      float acc[16];
+  for (int s0 = 0; s0 < p.B; s0 += p.sb) {
+    const int nsb = min(p.sb, p.B - s0);
+    for (int b0 = s0; b0 < s0 + nsb; b0 += kReduceNBB) {
+      const int nbb = min(kReduceNBB, s0 + nsb - b0);
+      // ū of the block straight from the partials: float4 loads, eight items in flight per thread
+      const int nv = DB / 4;
+      const size_t item4 = static_cast<size_t>(p.H) * p.d / 4;  // float4 stride between items
+      for (int i = tid; i < kReduceNBB * nv; i += kReduceThreads) {
+        const int bl = i / nv, c4 = i % nv;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (bl < nbb) {
+          const int lo = off[b0 + bl], hi = off[b0 + bl + 1];
+          const float4* src =
+              reinterpret_cast<const float4*>(p.U + (static_cast<size_t>(lo) * p.H + h) * p.d + c0) + c4;
+          int c = lo;
+          for (; c + 8 <= hi; c += 8) {
+            float4 v[8];
 #pragma unroll
-      for (int bl = 0; bl < 16; ++bl) acc[bl] = 0.f;
-      for (int i = g; i < DB; i += groups) {
-        const float w = ldw<WT>(W, static_cast<size_t>(c0 + i) * p.d + h * d_h + j);
+            for (int u = 0; u < 8; ++u) v[u] = __ldg(src + u * item4);
 #pragma unroll
-        for (int bl = 0; bl < 16; ++bl)
-          if (bl < nbb) acc[bl] = fmaf(ubar[bl * DB + i], w, acc[bl]);
+            for (int u = 0; u < 8; ++u) {
+              const float w = wts[c + u];
+              acc.x = fmaf(w, v[u].x, acc.x);
+              acc.y = fmaf(w, v[u].y, acc.y);
+              acc.z = fmaf(w, v[u].z, acc.z);
+              acc.w = fmaf(w, v[u].w, acc.w);
+            }
+            src += 8 * item4;
+          }
+          for (; c < hi; ++c, src += item4) {
+            const float4 v = __ldg(src);
+            const float w = wts[c];
+            acc.x = fmaf(w, v.x, acc.x);
+            acc.y = fmaf(w, v.y, acc.y);
+            acc.z = fmaf(w, v.z, acc.z);
+            acc.w = fmaf(w, v.w, acc.w);
+          }
+        }
+        *reinterpret_cast<float4*>(ubar + bl * DB + 4 * c4) = acc;
       }
+      __syncthreads();
+      // partial head output of the block: ū[bl, d-block] · W_KV[d-block rows, head-h columns]
+      float acc[kReduceNBB][VEC];
 #pragma unroll
-      for (int bl = 0; bl < 16; ++bl)
-        if (bl < nbb) red[(g * p.bb + bl) * d_h + j] = acc[bl];
+      for (int bl = 0; bl < kReduceNBB; ++bl)
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) acc[bl][v] = 0.f;
+      if (g < G) {
+        const WT* wp = W + static_cast<size_t>(c0) * p.d + h * d_h + cg * VEC;
+#pragma unroll 4
+        for (int i = g; i < DB; i += G) {
+          float w[VEC];
+          WVec<WT>::load(wp + static_cast<size_t>(i) * p.d, w);
+#pragma unroll
+          for (int bl = 0; bl < kReduceNBB; ++bl) {
+            const float u = ubar[bl * DB + i];
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) acc[bl][v] = fmaf(u, w[v], acc[bl][v]);
+          }
+        }
+      }
+      // reduce the row groups of a warp with shuffles, then across warps through shared memory
+#pragma unroll
+      for (int bl = 0; bl < kReduceNBB; ++bl)
+#pragma unroll
+        for (int v = 0; v < VEC; ++v)
+          for (int o = ncg; o < 32; o <<= 1) acc[bl][v] += __shfl_xor_sync(0xffffffffu, acc[bl][v], o);
+      if (lane < ncg && g < G) {
+#pragma unroll
+        for (int bl = 0; bl < kReduceNBB; ++bl)
+#pragma unroll
+          for (int v = 0; v < VEC; ++v) red[(warp * kReduceNBB + bl) * d_h + cg * VEC + v] = acc[bl][v];
+      }
+      __syncthreads();
+      const int nwarps = min(kReduceThreads / 32, (G + gpw - 1) / gpw);
+      for (int i = tid; i < nbb * d_h; i += kReduceThreads) {
+        float sum = 0.f;
+        for (int w2 = 0; w2 < nwarps; ++w2) sum += red[w2 * kReduceNBB * d_h + i];
+        part[(b0 - s0) * d_h + i] = sum;
+      }
+      __syncthreads();
     }
-    __syncthreads();
-    for (int i = tid; i < nbb * d_h; i += blockDim.x) {
-      float s = 0.f;
-      for (int gg = 0; gg < groups; ++gg) s += red[gg * p.bb * d_h + i];
-      part[i] = s;
-    }
-    // sum the NDB CTAs' products through distributed shared memory
+    // sum the NDB CTAs' products through distributed shared memory (fixed order)
     cluster_sync();
-    for (int i = tid; i < nbb * d_h; i += blockDim.x) {
+    for (int i = tid; i < nsb * d_h; i += kReduceThreads) {
       if (i % p.ndb != r) continue;
-      float s = 0.f;
-      for (int rr = 0; rr < p.ndb; ++rr) s += ld_cluster_f32(mapa_shared(part_base + 4u * i, rr));
+      float sum = 0.f;
+      for (int q = 0; q < p.ndb; ++q) sum += ld_cluster_f32(mapa_shared(part_base + 4u * i, q));
       const int bl = i / d_h, jj = i % d_h;
-      p.out[static_cast<size_t>(b0 + bl) * p.d + h * d_h + jj] = s;
+      p.out[static_cast<size_t>(s0 + bl) * p.d + h * d_h + jj] = sum;
     }
     cluster_sync();
   }
@@ -189,7 +274,8 @@ int pick_ndb(int d, int d_h) {
 cudaError_t launch_reduce_b(const DecodeArgs& a, const SplitWorkspace& ws, bool pdl, cudaStream_t st,
                             int* launches) {
   const int d_h = a.d / a.H;
-  if (d_h > 256) return cudaErrorNotSupported;
+  const int vec = (a.dtype == SLIM_BF16) ? 8 : 4;
+  if (d_h % vec || d_h / vec > 32 || (32 % (d_h / vec)) != 0) return cudaErrorNotSupported;
   ReduceBParams p;
   p.U = ws.U;
   p.m = ws.m;
@@ -198,28 +284,24 @@ cudaError_t launch_reduce_b(const DecodeArgs& a, const SplitWorkspace& ws, bool 
   p.w_kv = a.w_kv;
   p.out = a.out;
   p.lens = a.lens;
+  p.status = a.status;
   p.B = a.B;
   p.d = a.d;
   p.H = a.H;
   p.ndb = pick_ndb(a.d, d_h);
   p.max_items = ws.max_items;
   const int DB = a.d / p.ndb;
-  const int groups = 256 / d_h;
-  p.bb = 16;
-  size_t smem = 0;
-  for (;;) {
-    smem = sizeof(float) * (static_cast<size_t>(p.max_items) + static_cast<size_t>(p.bb) * DB +
-                            static_cast<size_t>(p.bb) * d_h + static_cast<size_t>(groups) * p.bb * d_h);
-    if (smem <= 200 * 1024 || p.bb == 1) break;
-    p.bb /= 2;
-  }
-  if (smem > 200 * 1024) return cudaErrorNotSupported;
+  if (DB % 4) return cudaErrorNotSupported;
+  p.sb = std::max(kReduceNBB, std::min(a.B, (32 * 1024) / (d_h * 4)) / kReduceNBB * kReduceNBB);
+  p.sb = std::min(p.sb, ((a.B + kReduceNBB - 1) / kReduceNBB) * kReduceNBB);
+  const size_t smem = reduce_smem_layout(p.max_items, DB, d_h, p.sb).total;
+  if (smem > 200u * 1024u) return cudaErrorNotSupported;
   auto kern = (a.dtype == SLIM_BF16) ? reduce_b_kernel<__nv_bfloat16> : reduce_b_kernel<float>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(a.H), static_cast<unsigned>(p.ndb), 1);
-  cfg.blockDim = dim3(256, 1, 1);
+  cfg.blockDim = dim3(kReduceThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];

@@ -70,6 +70,19 @@ bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uin
   return r == CUDA_SUCCESS;
 }
 
+bool encode_tmap_kslab(CUtensorMap* map, const void* base, uint64_t rows, int d, int box_blocks) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn || d % 64 || box_blocks < 1 || box_blocks > 256) return false;
+  cuuint64_t dims[3] = {64, rows, static_cast<cuuint64_t>(d / 64)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2u, 128};
+  cuuint32_t box[3] = {64, 16, static_cast<cuuint32_t>(box_blocks)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------------------------- workspace
 namespace {
 
@@ -123,6 +136,24 @@ SplitWorkspace carve(void* base, const WsLayout& w) {
 
 thread_local int g_last_launches = 0;
 
+// Measurement aid: event pairs recorded around the split kernel.
+struct TimingRing {
+  std::vector<cudaEvent_t> start, stop;
+  int next = 0, recorded = 0;
+};
+thread_local TimingRing g_timing;
+
+void timing_before(cudaStream_t st) {
+  if (g_timing.start.empty()) return;
+  cudaEventRecord(g_timing.start[g_timing.next], st);
+}
+void timing_after(cudaStream_t st) {
+  if (g_timing.start.empty()) return;
+  cudaEventRecord(g_timing.stop[g_timing.next], st);
+  g_timing.next = (g_timing.next + 1) % static_cast<int>(g_timing.start.size());
+  g_timing.recorded = std::min(g_timing.recorded + 1, static_cast<int>(g_timing.start.size()));
+}
+
 // ---------------------------------------------------------------------------- ordering table
 struct TuneKey {
   int dtype, B, d, H;
@@ -171,6 +202,35 @@ using namespace slim;
 extern "C" {
 
 int slim_version(void) { return 100; }
+
+int slim_timing_enable(int n) {
+  if (n < 0) return SLIM_EINVAL;
+  for (auto e : g_timing.start) cudaEventDestroy(e);
+  for (auto e : g_timing.stop) cudaEventDestroy(e);
+  g_timing = TimingRing{};
+  for (int i = 0; i < n; ++i) {
+    cudaEvent_t a, b;
+    if (cudaEventCreate(&a) != cudaSuccess || cudaEventCreate(&b) != cudaSuccess) {
+      cudaGetLastError();
+      return SLIM_ECUDA;
+    }
+    g_timing.start.push_back(a);
+    g_timing.stop.push_back(b);
+  }
+  return SLIM_OK;
+}
+
+int slim_timing_read(float* ms, int n) {
+  if (!ms || n < 0) return SLIM_EINVAL;
+  const int cnt = std::min(n, g_timing.recorded);
+  for (int i = 0; i < cnt; ++i) {
+    if (cudaEventElapsedTime(&ms[i], g_timing.start[i], g_timing.stop[i]) != cudaSuccess) {
+      cudaGetLastError();
+      return SLIM_ECUDA;
+    }
+  }
+  return cnt;
+}
 
 int slim_last_launch_count(void) { return g_last_launches; }
 
@@ -271,17 +331,12 @@ int slim_decode_step(const float* q, const void* k_new, void* Kcache, int32_t* l
   int launches = 0;
   cudaError_t e = cudaSuccess;
   if (v == SLIM_VARIANT_B) {
-    bool tc = false;
-    if (dtype == SLIM_BF16 && decode_b_tc_supported(B, d, H)) {
-      e = launch_decode_b_tc(a, ws, st, &launches);
-      tc = (e == cudaSuccess);
-      if (e == cudaErrorNotSupported) e = cudaSuccess;
-    }
-    if (!tc && e == cudaSuccess) {
-      if (!decode_b_simt_supported(B, d, H)) return SLIM_EUNSUPPORTED;
-      e = launch_decode_b_simt(a, ws, st, &launches);
-    }
-    if (e == cudaSuccess) e = launch_reduce_b(a, ws, /*pdl=*/true, st, &launches);
+    const bool tc = dtype == SLIM_BF16 && decode_b_tc_supported(B, d, H);
+    if (!tc && !decode_b_simt_supported(B, d, H)) return SLIM_EUNSUPPORTED;
+    timing_before(st);
+    e = tc ? launch_decode_b_tc(a, ws, st, &launches) : launch_decode_b_simt(a, ws, st, &launches);
+    timing_after(st);
+    if (e == cudaSuccess) e = launch_reduce_b(a, ws, /*pdl=*/g_timing.start.empty(), st, &launches);
   } else {
     if (!decode_a_supported(dtype, B, d, H)) return SLIM_EUNSUPPORTED;
     e = launch_decode_a(a, ws, st, &launches);

@@ -78,6 +78,10 @@ cudaError_t launch_rows_gemm(const void* A, const void* W, void* Y, const int32_
 bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
                          uint32_t box_inner, uint32_t box_outer, bool swizzle128);
 
+// K cache [rows][d] bf16 as a 3-D map {64 columns, rows, d/64 column blocks} with a box of
+// 64 x 16 x box_blocks, 128-byte swizzle: one load brings 16 rows of box_blocks column blocks.
+bool encode_tmap_kslab(CUtensorMap* map, const void* base, uint64_t rows, int d, int box_blocks);
+
 int num_sms();
 int max_smem_optin();
 

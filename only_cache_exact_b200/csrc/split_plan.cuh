@@ -27,14 +27,48 @@ struct SplitItem {
   int nb;    // attended rows of the sequence (incl. the appended one)
 };
 
-// Run by ONE full warp. s_nb, s_rows: [B]; s_off: [B+1] (shared memory).
-// n_slots must be >= B so that one chunk per sequence always fits.
-// report != 0: also writes the merge metadata and ORs length errors into *status.
-__device__ inline void plan_split(const int32_t* __restrict__ lens, int B, int64_t cap, int append, int n_slots,
-                                  int min_rows, int* s_nb, int* s_rows, int* s_off, int32_t* meta, int32_t* status,
-                                  bool report) {
+// Smallest chunk length C (a multiple of 16 rows, at least min_rows) such that
+// cutting every sequence into ceil(nb / C) chunks needs at most n_slots work
+// items. Bracketed first: C >= R / n_slots is necessary, and
+// C >= R / (n_slots - nonempty) is sufficient (ceil adds at most one chunk per
+// sequence), so the binary search usually runs a handful of steps. One warp.
+__device__ inline int plan_chunk(const int* s_nb, int B, long long n_slots, int min_rows, long long R, int nonempty,
+                                 int max_nb) {
   const int lane = threadIdx.x & 31;
-  int bad = 0;
+  const int cap16 = max((max_nb + 15) >> 4, 1);
+  int lo = (max(min_rows, 16) + 15) >> 4;
+  lo = max(lo, static_cast<int>((R + n_slots * 16 - 1) / (n_slots * 16)));
+  int hi = cap16;
+  if (n_slots > nonempty) {
+    const long long free_slots = n_slots - nonempty;
+    hi = min(hi, static_cast<int>((R + free_slots * 16 - 1) / (free_slots * 16)));
+  }
+  if (lo >= hi) return max(lo, 1) << 4;
+#pragma unroll 1
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    const int C = mid << 4;
+    int cnt = 0;
+    for (int b = lane; b < B; b += 32) cnt += (s_nb[b] + C - 1) / C;
+    cnt = warp_sum_int(cnt);
+    if (cnt <= n_slots) hi = mid; else lo = mid + 1;
+  }
+  return lo << 4;
+}
+
+// Run by ONE full warp. s_nb, s_rows: [B]; s_off: [B+1] (shared memory).
+// The work items are processed by n_groups CTA groups (CTAs or clusters),
+// group c taking items c, c + n_groups, ...; up to max_items items in total
+// (max_items >= B). The number of items per group is chosen among powers of
+// two to minimise the estimated longest group (rows of its items plus a fixed
+// per-item cost), which balances ragged batches.
+// report != 0: also writes the merge metadata and ORs length errors into *status.
+__device__ inline void plan_split(const int32_t* __restrict__ lens, int B, int64_t cap, int append, int n_groups,
+                                  int max_items, int min_rows, int* s_nb, int* s_rows, int* s_off, int32_t* meta,
+                                  int32_t* status, bool report) {
+  const int lane = threadIdx.x & 31;
+  int bad = 0, nonempty = 0, max_nb = 0;
+  long long R = 0;
   for (int b = lane; b < B; b += 32) {
     const int L = __ldg(lens + b);
     int nb;
@@ -48,29 +82,36 @@ __device__ inline void plan_split(const int32_t* __restrict__ lens, int B, int64
       nb = L + append;
     }
     s_nb[b] = nb;
+    R += nb;
+    nonempty += nb > 0;
+    max_nb = max(max_nb, nb);
     if (report) meta[2 + B + b] = (nb > 0 && append) ? kSeqAppend : 0;
   }
+  R = warp_sum_ll(R);
+  nonempty = warp_sum_int(nonempty);
+  max_nb = __reduce_max_sync(0xffffffffu, max_nb);
   bad = __reduce_or_sync(0xffffffffu, bad);
   if (report && lane == 0 && bad) atomicOr(status, bad);
   __syncwarp();
 
-  // Smallest chunk length C (a multiple of 16 rows, at least min_rows) such
-  // that cutting every sequence into ceil(nb / C) chunks needs no more than
-  // n_slots work items: this minimises the longest chunk, i.e. the step time.
-  int max_nb = 0;
-  for (int b = lane; b < B; b += 32) max_nb = max(max_nb, s_nb[b]);
-  max_nb = __reduce_max_sync(0xffffffffu, max_nb);
-  int lo = (max(min_rows, 16) + 15) >> 4, hi = max((max_nb + 15) >> 4, lo);
-#pragma unroll 1
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    const int C = mid << 4;
-    int cnt = 0;
-    for (int b = lane; b < B; b += 32) cnt += (s_nb[b] + C - 1) / C;
-    cnt = warp_sum_int(cnt);
-    if (cnt <= n_slots) hi = mid; else lo = mid + 1;
+  constexpr long long kItemCostRows = 128;  // epilogue + pipeline restart, in K rows
+  int chunk = 16;
+  long long best = -1;
+  for (int k = 1; static_cast<long long>(k) * n_groups <= max_items || k == 1; k <<= 1) {
+    const long long n_slots = max(static_cast<long long>(k) * n_groups, static_cast<long long>(nonempty));
+    if (n_slots > max_items && k > 1) break;
+    const int C = plan_chunk(s_nb, B, n_slots, min_rows, R, nonempty, max_nb);
+    int items = 0;
+    for (int b = lane; b < B; b += 32) items += (s_nb[b] + C - 1) / C;
+    items = warp_sum_int(items);
+    const long long per_group = (items + n_groups - 1) / n_groups;
+    const long long est = per_group * (C + kItemCostRows);
+    if (best < 0 || est < best) {
+      best = est;
+      chunk = C;
+    }
+    if (k > 64) break;
   }
-  const int chunk = lo << 4;
 
   int carry = 0;
   for (int base = 0; base < B; base += 32) {

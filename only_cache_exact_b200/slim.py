@@ -27,7 +27,7 @@ SLIM_AUTO, SLIM_VARIANT_A, SLIM_VARIANT_B = 0, 1, 2
 EXPORTS = [
     "slim_prefill_k", "slim_decode_workspace_bytes", "slim_decode_step", "slim_decode_step_host", "slim_tune",
     "slim_tune_record", "slim_select_variant", "slim_tune_clear", "slim_strerror", "slim_last_launch_count",
-    "slim_version",
+    "slim_version", "slim_timing_enable", "slim_timing_read",
 ]
 
 _vp, _i32, _i64, _sz, _f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
@@ -46,6 +46,8 @@ _SIGS = {
     "slim_strerror": (ctypes.c_char_p, [_i32]),
     "slim_last_launch_count": (_i32, []),
     "slim_version": (_i32, []),
+    "slim_timing_enable": (_i32, [_i32]),
+    "slim_timing_read": (_i32, [_vp, _i32]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -170,6 +172,18 @@ def slim_select_variant(dtype: int, B: int, d: int, H: int, T: int) -> int:
 
 def slim_tune_clear() -> None:
     _lib.slim_tune_clear()
+
+
+def slim_timing_enable(n: int) -> None:
+    _check(_lib.slim_timing_enable(int(n)), "slim_timing_enable")
+
+
+def slim_timing_read(n: int) -> list:
+    buf = (ctypes.c_float * max(n, 1))()
+    cnt = _lib.slim_timing_read(buf, int(n))
+    if cnt < 0:
+        raise SlimError(cnt, "slim_timing_read")
+    return [float(buf[i]) for i in range(cnt)]
 
 
 def raw_lib() -> ctypes.CDLL:
