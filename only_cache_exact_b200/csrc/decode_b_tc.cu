@@ -318,6 +318,21 @@ __global__ void __launch_bounds__(kTCThreads, 1)
     // ------------------------------------------------------------ score / softmax warps
     const int sw = warp - 6;  // heads sw, sw + 8, ... of this CTA
     const int gq = lane >> 2, tq = lane & 3;  // mma.sync fragment coordinates
+    // This lane's ldmatrix.x4 row address (relative to a K stage) for head k, row block rb,
+    // 16-column step ks: lanes 0-7 give rows 0-7 / columns 0-7, lanes 8-15 rows 8-15 /
+    // columns 0-7, lanes 16-23 rows 0-7 / columns 8-15, lanes 24-31 rows 8-15 / columns 8-15.
+    uint32_t a_off[HPW][TT / 16][DHB * 4];
+#pragma unroll
+    for (int k = 0; k < HPW; ++k)
+#pragma unroll
+      for (int rb = 0; rb < TT / 16; ++rb)
+#pragma unroll
+        for (int ks = 0; ks < DHB * 4; ++ks) {
+          const int row = rb * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
+          const int colk = (sw + kSoftmaxWarps * k) * DH + ks * 16 + (lane >> 4) * 8;
+          a_off[k][rb][ks] = static_cast<uint32_t>((row >> 4) * slab_bytes + (colk >> 6) * 2048 + (row & 15) * 128 +
+                                                   ((((colk & 63) >> 3) ^ (row & 7)) << 4));
+        }
     const uint32_t kbase = smem_u32(kst);
     const uint32_t pst_base = smem_u32(pst);
     const uint32_t alpha_base = smem_u32(alpha_s);
@@ -417,44 +432,57 @@ __global__ void __launch_bounds__(kTCThreads, 1)
         }
 
         const uint32_t kt = kbase + s * kstage_bytes;
+        // Phase 1: scores of every head of this warp, independent MMA chains
+        // interleaved; rows (16 rb + gq) and (16 rb + gq + 8) land in lanes tq == 0.
+        float sc[HPW][TT / 8];
+#pragma unroll
+        for (int rb = 0; rb < TT / 16; ++rb) {
+          float acc[HPW][4];
+#pragma unroll
+          for (int k = 0; k < HPW; ++k) acc[k][0] = acc[k][1] = acc[k][2] = acc[k][3] = 0.f;
+#pragma unroll
+          for (int ks = 0; ks < DHB * 4; ++ks) {
+#pragma unroll
+            for (int k = 0; k < HPW; ++k) {
+              if (sw + kSoftmaxWarps * k >= H_own) continue;
+              uint32_t a[4];
+              ldmatrix_x4(kt + a_off[k][rb][ks], a);
+              mma_16816_bf16(acc[k], a, bq[k][ks][0], bq[k][ks][1]);
+            }
+          }
+#pragma unroll
+          for (int k = 0; k < HPW; ++k) {
+            sc[k][2 * rb] = acc[k][0] + acc[k][1];
+            sc[k][2 * rb + 1] = acc[k][2] + acc[k][3];
+          }
+        }
+        // Phase 2: tile maxima of every head, shuffle trees interleaved
+        float mx[HPW];
+#pragma unroll
+        for (int k = 0; k < HPW; ++k) {
+          mx[k] = -INFINITY;
+#pragma unroll
+          for (int i = 0; i < TT / 8; ++i) {
+            const int trow = 8 * i + gq;  // (rb, half) = (i / 2, i % 2): row 16 rb + 8 half + gq
+            sc[k][i] = (tq == 0 && trow < nvalid) ? sc[k][i] * p.scale_log2 : -INFINITY;
+            mx[k] = fmaxf(mx[k], sc[k][i]);
+          }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+          for (int k = 0; k < HPW; ++k) mx[k] = fmaxf(mx[k], __shfl_xor_sync(0xffffffffu, mx[k], o));
+        // Phase 3: lazy running max, P to shared memory (and the cluster peers)
 #pragma unroll
         for (int k = 0; k < HPW; ++k) {
           const int hh = sw + kSoftmaxWarps * k;
           if (hh >= H_own) continue;
-          // scores of rows (16 rb + gq) and (16 rb + gq + 8) in lanes with tq == 0
-          float sc[TT / 8];
-#pragma unroll
-          for (int rb = 0; rb < TT / 16; ++rb) {
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-            // ldmatrix.x4: lanes 0-7 rows 0-7 / k 0-7, 8-15 rows 8-15 / k 0-7,
-            // 16-23 rows 0-7 / k 8-15, 24-31 rows 8-15 / k 8-15 of the 16x16 A tile
-            const int row = rb * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
-#pragma unroll
-            for (int ks = 0; ks < DHB * 4; ++ks) {
-              const int colk = hh * DH + ks * 16 + (lane >> 4) * 8;  // first column of this lane's 8x8 matrix
-              const uint32_t addr = kt + (row >> 4) * slab_bytes + (colk >> 6) * 2048 + (row & 15) * 128 +
-                                    ((((colk & 63) >> 3) ^ (row & 7)) << 4);
-              uint32_t a[4];
-              ldmatrix_x4(addr, a);
-              mma_16816_bf16(acc, a, bq[k][ks][0], bq[k][ks][1]);
-            }
-            sc[2 * rb] = acc[0] + acc[1];
-            sc[2 * rb + 1] = acc[2] + acc[3];
-          }
-          float mx = -INFINITY;
-#pragma unroll
-          for (int i = 0; i < TT / 8; ++i) {
-            const int trow = 8 * i + gq;  // (rb, half) = (i / 2, i % 2): row 16 rb + 8 half + gq
-            sc[i] = (tq == 0 && trow < nvalid) ? sc[i] * p.scale_log2 : -INFINITY;
-            mx = fmaxf(mx, sc[i]);
-          }
-          mx = warp_max(mx);
           float alpha = 1.f;
           if (t == 0) {
-            mref[k] = mx;
-          } else if (mx > mref[k] + kLazyRescaleLog2) {
-            alpha = exp2f(mref[k] - mx);
-            mref[k] = mx;
+            mref[k] = mx[k];
+          } else if (mx[k] > mref[k] + kLazyRescaleLog2) {
+            alpha = exp2f(mref[k] - mx[k]);
+            mref[k] = mx[k];
             lsum[k] *= alpha;
           }
           const int n = head0 + hh;
@@ -463,7 +491,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
 #pragma unroll
             for (int i = 0; i < TT / 8; ++i) {
               const int trow = 8 * i + gq;
-              const float pv = (trow < nvalid) ? exp2f(sc[i] - mref[k]) : 0.f;
+              const float pv = (trow < nvalid) ? exp2f(sc[k][i] - mref[k]) : 0.f;
               const __nv_bfloat16 pb = __float2bfloat16_rn(pv);
               lsum[k] += __bfloat162float(pb);
               const uint32_t off = static_cast<uint32_t>(s) * pstage_bytes +
