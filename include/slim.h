@@ -137,6 +137,29 @@ int slim_decode_step_host(const float* q_host, const void* k_new_host, void* Kca
                           float* out_host, void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream);
 
 /*
+ * slim_decode_step_noalloc — slim_decode_step without a caller workspace,
+ * for callers that cannot allocate device memory (code that must not call
+ * cudaMalloc, e.g. while a framework captures a CUDA graph or runs under a
+ * fixed memory plan). The paper has no counterpart: this is a packaging of
+ * the same step. Arguments and results are those of slim_decode_step minus
+ * `workspace`/`ws_bytes`; this call itself allocates nothing.
+ *
+ * Scratch: a buffer of SLIM_NOALLOC_SCRATCH_BYTES compiled into the library,
+ * present on every GPU that loads it until the process exits. Sizes whose
+ * slim_decode_workspace_bytes(...) exceeds it are rejected with
+ * SLIM_EWORKSPACE before anything is launched. The first call on a device
+ * looks up the buffer's device address (cudaGetSymbolAddress); make that
+ * first call outside any stream capture. Every call on a device shares the
+ * one buffer, which keeps the previous call's contents (the step needs no
+ * zeroed scratch), so calls that overlap on the GPU, e.g. on two streams,
+ * race with each other and must be serialised by the caller.
+ */
+#define SLIM_NOALLOC_SCRATCH_BYTES (32 * 1024 * 1024)
+int slim_decode_step_noalloc(const float* q, const void* k_new, void* Kcache, int32_t* lens, const void* W_KV,
+                             int dtype, int B, int d, int H, int64_t cap, int variant, int64_t t_hint, float* out,
+                             int32_t* dev_status, void* stream);
+
+/*
  * slim_tune — fills the SLIM_AUTO table for (dtype, B, d, H) by timing both
  * orderings, without append, at each attended length Ts[i] (1 <= Ts[i] <= cap)
  * with CUDA events on `stream`, `reps` repetitions each. It overwrites

@@ -27,7 +27,7 @@ SLIM_AUTO, SLIM_VARIANT_A, SLIM_VARIANT_B = 0, 1, 2
 EXPORTS = [
     "slim_prefill_k", "slim_decode_workspace_bytes", "slim_decode_step", "slim_decode_step_host", "slim_tune",
     "slim_tune_record", "slim_select_variant", "slim_tune_clear", "slim_strerror", "slim_last_launch_count",
-    "slim_version", "slim_timing_enable", "slim_timing_read",
+    "slim_version", "slim_timing_enable", "slim_timing_read", "slim_decode_step_noalloc",
 ]
 
 _vp, _i32, _i64, _sz, _f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
@@ -48,7 +48,10 @@ _SIGS = {
     "slim_version": (_i32, []),
     "slim_timing_enable": (_i32, [_i32]),
     "slim_timing_read": (_i32, [_vp, _i32]),
+    "slim_decode_step_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i64, _i32, _i64, _vp, _vp,
+                                        _vp]),
 }
+SLIM_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
     _fn.restype = _res
@@ -137,6 +140,18 @@ def slim_decode_step(q: torch.Tensor, k_new, Kcache: torch.Tensor, lens: torch.T
     _check(_lib.slim_decode_step(_ptr(q), _ptr(k_new), _ptr(Kcache), _ptr(lens), _ptr(W_KV), _DT[Kcache.dtype],
                                  B, d, H, cap, variant, t_hint, _ptr(out), _ptr(workspace), workspace.numel(),
                                  _ptr(status), _stream(stream)), "slim_decode_step")
+
+
+def slim_decode_step_noalloc(q: torch.Tensor, k_new, Kcache: torch.Tensor, lens: torch.Tensor, W_KV: torch.Tensor,
+                             H: int, out: torch.Tensor, status: torch.Tensor, variant: int = SLIM_AUTO,
+                             t_hint: int = 0, stream=None) -> None:
+    """slim_decode_step for callers that cannot allocate: scratch comes from a buffer built into the library."""
+    for t, nm in ((q, "q"), (Kcache, "Kcache"), (lens, "lens"), (W_KV, "W_KV"), (out, "out"), (status, "status")):
+        _cuda(t, nm)
+    B, cap, d = Kcache.shape
+    _check(_lib.slim_decode_step_noalloc(_ptr(q), _ptr(k_new), _ptr(Kcache), _ptr(lens), _ptr(W_KV),
+                                         _DT[Kcache.dtype], B, d, H, cap, variant, t_hint, _ptr(out), _ptr(status),
+                                         _stream(stream)), "slim_decode_step_noalloc")
 
 
 def slim_decode_step_host(q_host: torch.Tensor, k_new_host, Kcache: torch.Tensor, lens: torch.Tensor,
