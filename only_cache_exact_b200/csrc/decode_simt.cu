@@ -55,14 +55,14 @@ struct SimtParams {
 constexpr int kSimtRows = 8;
 
 // Shared memory of the SIMT decode kernels.
-__host__ __device__ inline size_t simt_smem_bytes(int d, int H, int B, bool with_v) {
+// (K and V tiles are staged in the cache's own element type, esize bytes.)
+__host__ __device__ inline size_t simt_smem_bytes(int d, int H, int B, bool with_v, int esize) {
+  const size_t tiles = static_cast<size_t>(kSimtRows) * d * esize * (with_v ? 2 : 1);
   size_t f = static_cast<size_t>(d)                      // q
-             + static_cast<size_t>(kSimtRows) * d        // K tile
-             + (with_v ? static_cast<size_t>(kSimtRows) * d : 0)  // V tile
              + static_cast<size_t>(with_v ? d : H * d)   // accumulator
              + 2 * static_cast<size_t>(H) * kSimtRows    // scores, p
              + 3 * static_cast<size_t>(H);               // m, l, alpha
-  return f * 4 + 3 * static_cast<size_t>(B + 1) * 4 + 16;
+  return f * 4 + ((tiles + 15) & ~size_t(15)) + 3 * static_cast<size_t>(B + 1) * 4 + 16;
 }
 
 template <typename KT, bool VARIANT_A>
@@ -70,15 +70,17 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(const SimtParams p) {
   extern __shared__ float sm[];
   const int d = p.d, H = p.H, d_h = d / H;
   float* q_s = sm;
-  float* ks = q_s + d;
-  float* vs = ks + kSimtRows * d;
-  float* acc = vs + (VARIANT_A ? kSimtRows * d : 0);
-  float* sc = acc + (VARIANT_A ? d : H * d);
+  float* acc = q_s + d;
+  float* sc_base = acc + (VARIANT_A ? d : H * d);
+  KT* ks = reinterpret_cast<KT*>(sc_base + 2 * H * kSimtRows + 3 * H);
+  KT* vs = ks + kSimtRows * d;
+  float* sc = sc_base;
   float* pm = sc + H * kSimtRows;
   float* mref = pm + H * kSimtRows;
   float* lsum = mref + H;
   float* alph = lsum + H;
-  int* s_nb = reinterpret_cast<int*>(alph + H);
+  int* s_nb = reinterpret_cast<int*>(
+      (reinterpret_cast<uintptr_t>(ks + kSimtRows * d * (VARIANT_A ? 2 : 1)) + 15) & ~uintptr_t(15));
   int* s_rows = s_nb + (p.B + 1);
   int* s_off = s_rows + (p.B + 1);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -109,16 +111,15 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(const SimtParams p) {
     for (int i = tid; i < kSimtRows * d; i += blockDim.x) {
       const int row = i / d, col = i % d;
       const int r = r_lo + row;
-      float kv = 0.f, vv = 0.f;
+      KT kv = from_f<KT>(0.f), vv = from_f<KT>(0.f);
       if (row < nvalid) {
         if (!VARIANT_A && p.append && r == nb_old) {
-          const KT x = kn[col];
-          kv = to_f<KT>(x);
-          static_cast<KT*>(p.kcache)[(static_cast<size_t>(b) * p.cap + r) * d + col] = x;
+          kv = kn[col];
+          static_cast<KT*>(p.kcache)[(static_cast<size_t>(b) * p.cap + r) * d + col] = kv;
         } else {
-          kv = to_f<KT>(K[static_cast<size_t>(r) * d + col]);
+          kv = K[static_cast<size_t>(r) * d + col];
         }
-        if (VARIANT_A) vv = to_f<KT>(V[static_cast<size_t>(r) * d + col]);
+        if (VARIANT_A) vv = V[static_cast<size_t>(r) * d + col];
       }
       ks[i] = kv;
       if (VARIANT_A) vs[i] = vv;
@@ -128,7 +129,7 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(const SimtParams p) {
     if (warp < kSimtRows) {
       for (int h = 0; h < H; ++h) {
         float s = 0.f;
-        for (int j = lane; j < d_h; j += 32) s = fmaf(q_s[h * d_h + j], ks[warp * d + h * d_h + j], s);
+        for (int j = lane; j < d_h; j += 32) s = fmaf(q_s[h * d_h + j], to_f<KT>(ks[warp * d + h * d_h + j]), s);
         s = warp_sum(s);
         if (lane == 0) sc[h * kSimtRows + warp] = (warp < nvalid) ? s * p.scale_log2 : -INFINITY;
       }
@@ -155,14 +156,14 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(const SimtParams p) {
       for (int col = tid; col < d; col += blockDim.x) {
         const int h = col / d_h;
         float x = acc[col] * alph[h];
-        for (int t = 0; t < kSimtRows; ++t) x = fmaf(pm[h * kSimtRows + t], vs[t * d + col], x);
+        for (int t = 0; t < kSimtRows; ++t) x = fmaf(pm[h * kSimtRows + t], to_f<KT>(vs[t * d + col]), x);
         acc[col] = x;
       }
     } else {
       for (int i = tid; i < H * d; i += blockDim.x) {
         const int h = i / d, col = i % d;
         float x = acc[i] * alph[h];
-        for (int t = 0; t < kSimtRows; ++t) x = fmaf(pm[h * kSimtRows + t], ks[t * d + col], x);
+        for (int t = 0; t < kSimtRows; ++t) x = fmaf(pm[h * kSimtRows + t], to_f<KT>(ks[t * d + col]), x);
         acc[i] = x;
       }
     }
@@ -288,7 +289,7 @@ SimtParams make_simt(const DecodeArgs& a, const SplitWorkspace& ws, bool variant
 template <bool VA>
 cudaError_t launch_simt(const DecodeArgs& a, const SplitWorkspace& ws, cudaStream_t st) {
   const SimtParams p = make_simt(a, ws, VA);
-  const size_t smem = simt_smem_bytes(a.d, a.H, a.B, VA);
+  const size_t smem = simt_smem_bytes(a.d, a.H, a.B, VA, a.dtype == SLIM_BF16 ? 2 : 4);
   if (smem > static_cast<size_t>(max_smem_optin())) return cudaErrorNotSupported;
   auto kern = (a.dtype == SLIM_BF16) ? decode_simt_kernel<__nv_bfloat16, VA> : decode_simt_kernel<float, VA>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -299,7 +300,7 @@ cudaError_t launch_simt(const DecodeArgs& a, const SplitWorkspace& ws, cudaStrea
 }  // namespace
 
 bool decode_b_simt_supported(int B, int d, int H) {
-  return simt_smem_bytes(d, H, B, false) <= static_cast<size_t>(max_smem_optin());
+  return simt_smem_bytes(d, H, B, false, 2) <= static_cast<size_t>(max_smem_optin());
 }
 
 cudaError_t launch_decode_b_simt(const DecodeArgs& a, const SplitWorkspace& ws, cudaStream_t st, int* launches) {
@@ -311,8 +312,7 @@ cudaError_t launch_decode_b_simt(const DecodeArgs& a, const SplitWorkspace& ws, 
 cudaError_t launch_reduce_a(const DecodeArgs& a, const SplitWorkspace& ws, cudaStream_t st, int* launches);
 
 bool decode_a_supported(int dtype, int B, int d, int H) {
-  (void)dtype;
-  return simt_smem_bytes(d, H, B, true) <= static_cast<size_t>(max_smem_optin());
+  return simt_smem_bytes(d, H, B, true, dtype == SLIM_BF16 ? 2 : 4) <= static_cast<size_t>(max_smem_optin());
 }
 
 cudaError_t launch_rows_gemm(const void* A, const void* W, void* Y, const int32_t* lens, int rows_extra, int dtype,
@@ -352,7 +352,8 @@ cudaError_t launch_decode_a(const DecodeArgs& a, const SplitWorkspace& ws, cudaS
     if (e != cudaSuccess) return e;
     if (launches) ++*launches;
   }
-  e = launch_rows_gemm_any(a.kcache, a.w_kv, ws.vbuf, a.lens, app, a.dtype, a.B, a.d, a.cap, st, launches);
+  e = launch_rows_gemm_any(a.kcache, a.w_kv, ws.vbuf, a.lens, app, a.dtype, a.B, a.d, a.cap, a.status, st,
+                           launches);
   if (e != cudaSuccess) return e;
   e = launch_simt<true>(a, ws, st);
   if (e != cudaSuccess) return e;

@@ -1,10 +1,188 @@
-// Prompt-phase projection K = X·W_K (and V = K·W_KV rows for ordering (a)):
-// length bookkeeping after the projection kernels.
+// Row GEMM Y = A·W on tcgen05 tensor cores (bf16 in, fp32 accumulation, bf16 out).
+//
+// Two uses (Slim Attention article, section "K-Cache is All You Need"):
+//   * prompt phase: K = X·W_K for n new tokens of every sequence, written to
+//     cache rows lens[b] .. lens[b]+n-1 (V is not computed);
+//   * ordering (a) of the generation phase: V = K·W_KV for the attended rows
+//     of every sequence, written to a V scratch with the cache's layout.
+// A CTA computes a 128-row x 256-column tile of one sequence. Warp 0 issues
+// TMA loads (A: 128 rows x 64 columns, K-major, 128-byte swizzle; W: 64 rows
+// x 256 columns as four MN-major 64-column blocks) into a 4-stage ring; warp
+// 1 issues tcgen05.mma M=128 N=256 K=16 into 256 TMEM columns; warps 2..5
+// convert the accumulator rows to bf16 and store them.
 #include <cuda_bf16.h>
 
 #include "ptx.cuh"
 
 namespace slim {
+
+namespace {
+
+constexpr int kBM = 128, kBN = 256, kBK = 64, kStages = 4;
+constexpr int kGemmThreads = 192;
+constexpr uint32_t kAStage = kBM * kBK * 2;  // 16 KB
+constexpr uint32_t kBStage = kBK * kBN * 2;  // 32 KB
+constexpr uint32_t kGemmSmem = kStages * (kAStage + kBStage) + 1024 + 256;
+
+struct GemmParams {
+  __nv_bfloat16* Y;
+  const int32_t* lens;
+  int B, n, d, mode, extra;  // mode 0: prompt rows of X; mode 1: attended cache rows
+  int64_t cap;
+  int64_t a_rows_per_seq;    // rows per sequence in the A tensor map (n or cap)
+};
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap wmap,
+                   const GemmParams p, int32_t* status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* as = smem;
+  uint8_t* bs = smem + kStages * kAStage;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * (kAStage + kBStage));
+  uint64_t* empty = full + kStages;
+  uint64_t* accfull = empty + kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accfull + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * kBN, m0 = blockIdx.y * kBM, b = blockIdx.z;
+
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&amap);
+    tma_prefetch_desc(&wmap);
+  } else if (warp == 1) {
+    if (lane == 0) {
+      for (int s = 0; s < kStages; ++s) {
+        mbar_init(&full[s], 1);
+        mbar_init(&empty[s], 1);
+      }
+      mbar_init(accfull, 1);
+      fence_barrier_init();
+    }
+    __syncwarp();
+    tmem_alloc(tmem_slot, kBN);
+    tmem_relinquish();
+  }
+  pdl_wait_primary();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // rows of this sequence to produce and where they go
+  const int L = __ldg(p.lens + b);
+  int nrows;
+  int64_t out_row0;
+  if (p.mode == 0) {
+    nrows = (L < 0 || static_cast<int64_t>(L) + p.n > p.cap) ? 0 : p.n;
+    out_row0 = static_cast<int64_t>(b) * p.cap + L;
+  } else {
+    const int64_t v = static_cast<int64_t>(L) + p.extra;
+    nrows = (L < 0 || v > p.cap) ? 0 : static_cast<int>(v);
+    out_row0 = static_cast<int64_t>(b) * p.cap;
+  }
+  const bool active = m0 < nrows;
+  const int nk = p.d / kBK;
+
+  if (warp == 0) {
+    if (lane == 0 && active) {
+      const uint64_t pol_a = l2_policy_evict_first();
+      const uint64_t pol_w = l2_policy_evict_last();
+      const int a_row = static_cast<int>(static_cast<int64_t>(b) * p.a_rows_per_seq + m0);
+      int k = 0;
+      for (; k < nk; ++k) {
+        const int s = k % kStages;
+        const uint32_t ph = static_cast<uint32_t>(k / kStages) & 1u;
+        if (k >= kStages && !mbar_wait(&empty[s], ph ^ 1u, status)) break;
+        mbar_arrive_expect_tx(&full[s], kAStage + kBStage);
+        tma_load_2d(as + s * kAStage, &amap, k * kBK, a_row, &full[s], pol_a);
+        tma_load_3d(bs + s * kBStage, &wmap, 0, k * kBK, n0 / 64, &full[s], pol_w);
+      }
+      for (int t = max(0, k - kStages); t < k; ++t)
+        mbar_wait(&full[t % kStages], static_cast<uint32_t>(t / kStages) & 1u, status);
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && active) {
+      const uint32_t idesc = idesc_bf16_f32(kBM, kBN, 0u, 1u);
+      const uint32_t abase = smem_u32(as), bbase = smem_u32(bs);
+      int k = 0;
+      for (; k < nk; ++k) {
+        const int s = k % kStages;
+        const uint32_t ph = static_cast<uint32_t>(k / kStages) & 1u;
+        if (!mbar_wait(&full[s], ph, status)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          // A: K-major, 128-byte swizzle, 8-row groups 1024 B apart; a 16-column step is 32 B.
+          const uint64_t ad = smem_desc(abase + s * kAStage + kk * 32, 16, 1024, kLayoutSW128);
+          // W: MN-major, 64-column blocks 64 rows x 128 B (8 KB) apart, 8-row groups 1024 B apart.
+          const uint64_t bd = smem_desc(bbase + s * kBStage + kk * 16 * 128, kBK * 128, 1024, kLayoutSW128);
+          umma_f16(tmem, ad, bd, idesc, (k > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&empty[s]);
+      }
+      umma_commit(accfull);
+      mbar_wait(accfull, 0, status);
+    }
+  } else if (active) {
+    // epilogue: TMEM lane = tile row, columns = output columns
+    const int quarter = warp & 3;
+    const int r = m0 + quarter * 32 + lane;
+    if (__all_sync(0xffffffffu, mbar_wait(accfull, 0, status))) {
+      tc_fence_after();
+      __nv_bfloat16* dst = p.Y + (out_row0 + r) * p.d + n0;
+      for (int c = 0; c < kBN; c += 16) {
+        float v[16];
+        tmem_ld16(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + c, v);
+        tmem_wait_ld();
+        if (r < nrows) {
+          uint4 o0, o1;
+          o0.x = pack_bf16x2(v[0], v[1]);
+          o0.y = pack_bf16x2(v[2], v[3]);
+          o0.z = pack_bf16x2(v[4], v[5]);
+          o0.w = pack_bf16x2(v[6], v[7]);
+          o1.x = pack_bf16x2(v[8], v[9]);
+          o1.y = pack_bf16x2(v[10], v[11]);
+          o1.z = pack_bf16x2(v[12], v[13]);
+          o1.w = pack_bf16x2(v[14], v[15]);
+          *reinterpret_cast<uint4*>(dst + c) = o0;
+          *reinterpret_cast<uint4*>(dst + c + 8) = o1;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kBN);
+  }
+}
+
+// W [d rows][d cols] bf16 viewed as {64 columns, d rows, d/64 column blocks}; box 64 x 64 x 4.
+bool encode_wmap(CUtensorMap* map, const void* W, int d) {
+  return encode_tmap_3d_bf16(map, W, 64, static_cast<uint64_t>(d), static_cast<uint64_t>(d / 64),
+                             static_cast<uint64_t>(d) * 2u, 128u, 64, kBK, kBN / 64);
+}
+
+cudaError_t launch_gemm(const void* A, uint64_t a_rows_total, int64_t a_rows_per_seq, const void* W, void* Y,
+                        const int32_t* lens, int B, int n, int d, int64_t cap, int mode, int extra, int grid_rows,
+                        int32_t* status, cudaStream_t st, int* launches) {
+  CUtensorMap amap, wmap;
+  if (!encode_tmap_2d_bf16(&amap, A, static_cast<uint64_t>(d), a_rows_total, static_cast<uint64_t>(d) * 2u, kBK,
+                           kBM, true) ||
+      !encode_wmap(&wmap, W, d))
+    return cudaErrorInvalidValue;
+  GemmParams p{static_cast<__nv_bfloat16*>(Y), lens, B, n, d, mode, extra, cap, a_rows_per_seq};
+  cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem);
+  if (e != cudaSuccess) return e;
+  gemm_tc_kernel<<<dim3(d / kBN, (grid_rows + kBM - 1) / kBM, B), kGemmThreads, kGemmSmem, st>>>(amap, wmap, p,
+                                                                                                 status);
+  e = cudaGetLastError();
+  if (e == cudaSuccess && launches) ++*launches;
+  return e;
+}
+
+}  // namespace
 
 // lens[b] += n where the n new rows fitted (lens[b] + n <= cap); otherwise the
 // projection kernels skipped the sequence and the status word records why.
@@ -27,19 +205,20 @@ cudaError_t launch_advance_lens(int32_t* lens, int B, int n, int64_t cap, int32_
   return e;
 }
 
-bool gemm_tc_supported(int d) {
-  (void)d;
-  return false;
+bool gemm_tc_supported(int d) { return d >= kBN && d % kBN == 0; }
+
+cudaError_t launch_prefill_tc(const void* X, const void* W, void* kcache, const int32_t* lens, int B, int n, int d,
+                              int64_t cap, int32_t* status, cudaStream_t st, int* launches) {
+  if (!gemm_tc_supported(d)) return cudaErrorNotSupported;
+  return launch_gemm(X, static_cast<uint64_t>(B) * n, n, W, kcache, lens, B, n, d, cap, 0, 0, n, status, st,
+                     launches);
 }
 
-cudaError_t launch_prefill_tc(const void*, const void*, void*, const int32_t*, int, int, int, int64_t, cudaStream_t,
-                              int*) {
-  return cudaErrorNotSupported;
-}
-
-cudaError_t launch_rows_gemm_tc(const void*, const void*, void*, const int32_t*, int, int, int, int64_t,
-                                cudaStream_t, int*) {
-  return cudaErrorNotSupported;
+cudaError_t launch_rows_gemm_tc(const void* A, const void* W, void* Y, const int32_t* lens, int rows_extra, int B,
+                                int d, int64_t cap, int32_t* status, cudaStream_t st, int* launches) {
+  if (!gemm_tc_supported(d)) return cudaErrorNotSupported;
+  return launch_gemm(A, static_cast<uint64_t>(B) * cap, cap, W, Y, lens, B, 0, d, cap, 1, rows_extra,
+                     static_cast<int>(cap), status, st, launches);
 }
 
 }  // namespace slim

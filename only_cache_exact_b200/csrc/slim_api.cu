@@ -70,17 +70,24 @@ bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uin
   return r == CUDA_SUCCESS;
 }
 
-bool encode_tmap_kslab(CUtensorMap* map, const void* base, uint64_t rows, int d, int box_blocks) {
+bool encode_tmap_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
+                         uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2) {
   EncodeTiledFn fn = get_encode_fn();
-  if (!fn || d % 64 || box_blocks < 1 || box_blocks > 256) return false;
-  cuuint64_t dims[3] = {64, rows, static_cast<cuuint64_t>(d / 64)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2u, 128};
-  cuuint32_t box[3] = {64, 16, static_cast<cuuint32_t>(box_blocks)};
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1, s2};
+  cuuint32_t box[3] = {b0, b1, b2};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+bool encode_tmap_kslab(CUtensorMap* map, const void* base, uint64_t rows, int d, int box_blocks) {
+  if (d % 64 || box_blocks < 1 || box_blocks > 256) return false;
+  return encode_tmap_3d_bf16(map, base, 64, rows, static_cast<uint64_t>(d / 64), static_cast<uint64_t>(d) * 2u, 128,
+                             64, 16, static_cast<uint32_t>(box_blocks));
 }
 
 // ---------------------------------------------------------------------------- workspace
@@ -180,17 +187,18 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 cudaError_t launch_prefill_simt(const void* X, const void* W, void* kcache, const int32_t* lens, int dtype, int B,
                                 int n, int d, int64_t cap, cudaStream_t st, int* launches);
 cudaError_t launch_prefill_tc(const void* X, const void* W, void* kcache, const int32_t* lens, int B, int n, int d,
-                              int64_t cap, cudaStream_t st, int* launches);
+                              int64_t cap, int32_t* status, cudaStream_t st, int* launches);
 cudaError_t launch_rows_gemm_tc(const void* A, const void* W, void* Y, const int32_t* lens, int rows_extra, int B,
-                                int d, int64_t cap, cudaStream_t st, int* launches);
+                                int d, int64_t cap, int32_t* status, cudaStream_t st, int* launches);
 bool gemm_tc_supported(int d);
 cudaError_t launch_advance_lens(int32_t* lens, int B, int n, int64_t cap, int32_t* status, cudaStream_t st,
                                 int* launches);
 
 cudaError_t launch_rows_gemm_any(const void* A, const void* W, void* Y, const int32_t* lens, int rows_extra,
-                                 int dtype, int B, int d, int64_t cap, cudaStream_t st, int* launches) {
+                                 int dtype, int B, int d, int64_t cap, int32_t* status, cudaStream_t st,
+                                 int* launches) {
   if (dtype == SLIM_BF16 && gemm_tc_supported(d))
-    return launch_rows_gemm_tc(A, W, Y, lens, rows_extra, B, d, cap, st, launches);
+    return launch_rows_gemm_tc(A, W, Y, lens, rows_extra, B, d, cap, status, st, launches);
   return launch_rows_gemm(A, W, Y, lens, rows_extra, dtype, B, d, cap, st, launches);
 }
 
@@ -259,7 +267,7 @@ int slim_prefill_k(const void* X, const void* W_K, void* Kcache, int32_t* lens, 
   int launches = 0;
   cudaError_t e;
   if (dtype == SLIM_BF16 && gemm_tc_supported(d) && aligned(X, 16) && aligned(W_K, 16) && aligned(Kcache, 16))
-    e = launch_prefill_tc(X, W_K, Kcache, lens, B, n, d, cap, st, &launches);
+    e = launch_prefill_tc(X, W_K, Kcache, lens, B, n, d, cap, dev_status, st, &launches);
   else
     e = launch_prefill_simt(X, W_K, Kcache, lens, dtype, B, n, d, cap, st, &launches);
   if (e == cudaSuccess) e = launch_advance_lens(lens, B, n, cap, dev_status, st, &launches);

@@ -70,7 +70,8 @@ cudaError_t launch_reduce_a(const DecodeArgs& a, const SplitWorkspace& ws, cudaS
 // Row-wise GEMM used by variant (a): Y[b][t] = K[b][t]·W for t < lens[b] (+append) rows of each sequence.
 // _any picks the tcgen05 kernel for bf16 shapes it supports, else the CUDA-core one.
 cudaError_t launch_rows_gemm_any(const void* A, const void* W, void* Y, const int32_t* lens, int rows_extra,
-                                 int dtype, int B, int d, int64_t cap, cudaStream_t st, int* launches);
+                                 int dtype, int B, int d, int64_t cap, int32_t* status, cudaStream_t st,
+                                 int* launches);
 cudaError_t launch_rows_gemm(const void* A, const void* W, void* Y, const int32_t* lens, int rows_extra, int dtype,
                              int B, int d, int64_t cap, cudaStream_t st, int* launches);
 
@@ -78,6 +79,10 @@ cudaError_t launch_rows_gemm(const void* A, const void* W, void* Y, const int32_
 bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
                          uint32_t box_inner, uint32_t box_outer, bool swizzle128);
 
+// General 3-D bf16 tiled map: dims {d0, d1, d2} (d0 innermost, contiguous), byte strides s1, s2 of
+// dims 1 and 2, box {b0, b1, b2}, 128-byte swizzle (b0 * 2 must be <= 128).
+bool encode_tmap_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
+                         uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2);
 // K cache [rows][d] bf16 as a 3-D map {64 columns, rows, d/64 column blocks} with a box of
 // 64 x 16 x box_blocks, 128-byte swizzle: one load brings 16 rows of box_blocks column blocks.
 bool encode_tmap_kslab(CUtensorMap* map, const void* base, uint64_t rows, int d, int box_blocks);

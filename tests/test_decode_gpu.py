@@ -209,3 +209,30 @@ def test_bench_workload_sampled(S):
     got = g.step(S.SLIM_VARIANT_B)
     _check_bf16(got[[0, 7]], oracle_out(c, [0, 7]), c.H)
     assert np.all(np.isfinite(got))
+
+
+def test_bf16_prefill_d4096_tensor_core_gemm(S):
+    """tcgen05 GEMM path: K = X·W_K for 300 rows at d=4096, two sequences at different offsets."""
+    d, n = 4096, 300
+    w = synth.make_weights(d, 2, "bf16")
+    X = synth.make_tokens(n, d, 2, 0, "bf16")
+    K = torch.zeros(2, 700, d, dtype=torch.bfloat16, device="cuda")
+    lens = torch.tensor([5, 390], dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    Xt = synth.to_storage(X, "bf16").cuda()
+    S.slim_prefill_k(torch.stack([Xt, Xt]), synth.to_storage(w.W_K, "bf16").cuda(), K, lens, status)
+    torch.cuda.synchronize()
+    ref = X @ w.W_K
+    for b, off in ((0, 5), (1, 390)):
+        got = K[b, off:off + n].float().cpu().double().numpy()
+        rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+        assert rel <= 4e-3, rel
+    # rows outside the written range are untouched
+    assert float(K[0, :5].abs().max()) == 0.0 and float(K[1, 390 + n:].abs().max()) == 0.0
+    assert lens.cpu().tolist() == [305, 690] and int(status.item()) == 0
+
+
+def test_ordering_a_d4096(S):
+    c = make_case(4096, 32, lens=[200, 37], cap=300, seed=12)
+    g = GpuState(c, S)
+    _check_bf16(g.step(S.SLIM_VARIANT_A), oracle_out(c), c.H)
