@@ -24,15 +24,20 @@
 //   warps 2..5   correction and epilogue: the lazy online-softmax rescale of
 //                the accumulator rows whose max grew by more than 2^8, and
 //                TMEM -> partials in global memory.
-//   warps 6..13  scores: per head, q_h·K_t for 16 rows at a time with warp
-//                mma.sync (q split into bf16 high and low parts, fp32
-//                accumulation), running max, P in bf16 to shared memory and to
-//                the other CTAs of the cluster (distributed shared memory).
+//   warps 6..13  scores: per head, q_h·K_t on the CUDA cores, one K row per
+//                lane (16-byte loads from the swizzled stage, q broadcast from
+//                shared memory, fp32 accumulation), running max, P in bf16 to
+//                shared memory and to the other CTAs of the cluster
+//                (distributed shared memory). The tensor pipe is left to the
+//                P·K MMAs.
 // Every mbarrier wait is bounded; a timeout sets SLIM_DEV_TIMEOUT and the
 // kernel drains its copies and MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <map>
+#include <mutex>
+#include <utility>
 
 #include "split_plan.cuh"
 
@@ -267,7 +272,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
       for (int t = 0; t < nt; ++t, ++g) {
         const int s = g % stages;
         const uint32_t ph = static_cast<uint32_t>(g / stages) & 1u;
-        if (!__all_sync(0xffffffffu, mbar_wait(&pfull[s], ph, p.status))) {
+        if (!__all_sync(0xffffffffu, mbar_wait<(CL > 1)>(&pfull[s], ph, p.status))) {
           ok = false;
           break;
         }
@@ -300,14 +305,19 @@ __global__ void __launch_bounds__(kTCThreads, 1)
       if (!__all_sync(0xffffffffu, mbar_wait(accfull, static_cast<uint32_t>(ii) & 1u, p.status))) break;
       tc_fence_after();
       float* dst = p.ws_U + (static_cast<size_t>(item) * p.H + n) * p.d + col0 + 512 * hf;
-      for (int c = 0; c < hcols; c += 16) {
-        float v[16];
-        tmem_ld16(tbase + c, v);
+      // four 16-column loads in flight per wait (hcols and my_cols are multiples of 64)
+      for (int c = 0; c < hcols; c += 64) {
+        float v[4][16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) tmem_ld16(tbase + c + 16 * j, v[j]);
         tmem_wait_ld();
         if (n < p.H && c < my_cols) {
 #pragma unroll
-          for (int i = 0; i < 16; i += 4)
-            *reinterpret_cast<float4*>(dst + c + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+          for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int i = 0; i < 16; i += 4)
+              *reinterpret_cast<float4*>(dst + c + 16 * j + i) =
+                  make_float4(v[j][i], v[j][i + 1], v[j][i + 2], v[j][i + 3]);
         }
       }
       tc_fence_before();
@@ -317,22 +327,9 @@ __global__ void __launch_bounds__(kTCThreads, 1)
   } else {
     // ------------------------------------------------------------ score / softmax warps
     const int sw = warp - 6;  // heads sw, sw + 8, ... of this CTA
-    const int gq = lane >> 2, tq = lane & 3;  // mma.sync fragment coordinates
-    // This lane's ldmatrix.x4 row address (relative to a K stage) for head k, row block rb,
-    // 16-column step ks: lanes 0-7 give rows 0-7 / columns 0-7, lanes 8-15 rows 8-15 /
-    // columns 0-7, lanes 16-23 rows 0-7 / columns 8-15, lanes 24-31 rows 8-15 / columns 8-15.
-    uint32_t a_off[HPW][TT / 16][DHB * 4];
-#pragma unroll
-    for (int k = 0; k < HPW; ++k)
-#pragma unroll
-      for (int rb = 0; rb < TT / 16; ++rb)
-#pragma unroll
-        for (int ks = 0; ks < DHB * 4; ++ks) {
-          const int row = rb * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
-          const int colk = (sw + kSoftmaxWarps * k) * DH + ks * 16 + (lane >> 4) * 8;
-          a_off[k][rb][ks] = static_cast<uint32_t>((row >> 4) * slab_bytes + (colk >> 6) * 2048 + (row & 15) * 128 +
-                                                   ((((colk & 63) >> 3) ^ (row & 7)) << 4));
-        }
+    constexpr int HPP = 32 / TT;                  // heads per pass (one row per lane)
+    constexpr int NPASS = (HPW + HPP - 1) / HPP;  // passes over this warp's heads
+    const int row = lane % TT, hslot = lane / TT;
     const uint32_t kbase = smem_u32(kst);
     const uint32_t pst_base = smem_u32(pst);
     const uint32_t alpha_base = smem_u32(alpha_s);
@@ -343,16 +340,17 @@ __global__ void __launch_bounds__(kTCThreads, 1)
       const int nt = tiles_of(it);
       const int b = it.b;
       const int nb_old = it.nb - p.append;  // rows holding cached keys
-      // q of this warp's heads: to shared memory, then B fragments (column 0 = bf16 high part,
-      // column 1 = bf16 low part of q, other columns zero)
-      uint32_t bq[HPW][DHB * 4][2];
-      float mref[HPW], lsum[HPW];
+      // q of this warp's heads to shared memory (read back as broadcasts)
+      float mref[NPASS], lsum[NPASS];  // running max and sum of this lane's head in each pass
+#pragma unroll
+      for (int ps = 0; ps < NPASS; ++ps) {
+        mref[ps] = -INFINITY;
+        lsum[ps] = 0.f;
+      }
       __syncwarp();
 #pragma unroll
       for (int k = 0; k < HPW; ++k) {
         const int hh = sw + kSoftmaxWarps * k;
-        mref[k] = -INFINITY;
-        lsum[k] = 0.f;
         if (hh < H_own) {
           const float* src = p.q + static_cast<size_t>(b) * p.d + col0 + hh * DH;
           for (int i = lane; i < DH / 4; i += 32)
@@ -360,29 +358,6 @@ __global__ void __launch_bounds__(kTCThreads, 1)
         }
       }
       __syncwarp();
-#pragma unroll
-      for (int k = 0; k < HPW; ++k) {
-        const int hh = sw + kSoftmaxWarps * k;
-#pragma unroll
-        for (int ks = 0; ks < DHB * 4; ++ks) {
-          uint32_t v0 = 0, v1 = 0;
-          if (hh < H_own && gq < 2) {
-            const float* qc = q_s + hh * DH + ks * 16 + 2 * tq;
-            const float x0 = qc[0], x1 = qc[1], x8 = qc[8], x9 = qc[9];
-            if (gq == 0) {
-              v0 = pack_bf16x2(x0, x1);
-              v1 = pack_bf16x2(x8, x9);
-            } else {
-              v0 = pack_bf16x2(x0 - __bfloat162float(__float2bfloat16_rn(x0)),
-                               x1 - __bfloat162float(__float2bfloat16_rn(x1)));
-              v1 = pack_bf16x2(x8 - __bfloat162float(__float2bfloat16_rn(x8)),
-                               x9 - __bfloat162float(__float2bfloat16_rn(x9)));
-            }
-          }
-          bq[k][ks][0] = v0;
-          bq[k][ks][1] = v1;
-        }
-      }
 
       for (int t = 0; t < nt; ++t, ++g) {
         const int s = g % stages;
@@ -426,83 +401,80 @@ __global__ void __launch_bounds__(kTCThreads, 1)
         }
 
         // P stage s is free once the MMAs that read it (tile g - stages) finished in every CTA.
-        if (g >= stages && !__all_sync(0xffffffffu, mbar_wait(&pempty[s], ph ^ 1u, p.status))) {
+        if (g >= stages && !__all_sync(0xffffffffu, mbar_wait<(CL > 1)>(&pempty[s], ph ^ 1u, p.status))) {
           ok = false;
           break;
         }
 
         const uint32_t kt = kbase + s * kstage_bytes;
-        // Phase 1: scores of every head of this warp, independent MMA chains
-        // interleaved; rows (16 rb + gq) and (16 rb + gq + 8) land in lanes tq == 0.
-        float sc[HPW][TT / 8];
+        // Phase 1: scores on the CUDA cores (the tensor pipe is left to the P·K MMAs).
+        // Lane -> (row, head slot): row = lane % TT, and with TT = 16 the two half-warps
+        // take alternate heads. A lane reads its row's d_h columns of the head once
+        // (16-byte loads from the swizzled stage, conflict-free), q as broadcasts, and
+        // accumulates in fp32.
+        float sc[NPASS];
 #pragma unroll
-        for (int rb = 0; rb < TT / 16; ++rb) {
-          float acc[HPW][4];
+        for (int ps = 0; ps < NPASS; ++ps) {
+          const int k = ps * HPP + hslot;
+          const int hh = sw + kSoftmaxWarps * k;
+          float a0 = 0.f, a1 = 0.f;
+          if (k < HPW && hh < H_own) {
+            const uint32_t rbase = kt + (row >> 4) * slab_bytes + (row & 15) * 128;
+            const float4* qv = reinterpret_cast<const float4*>(q_s + hh * DH);
 #pragma unroll
-          for (int k = 0; k < HPW; ++k) acc[k][0] = acc[k][1] = acc[k][2] = acc[k][3] = 0.f;
-#pragma unroll
-          for (int ks = 0; ks < DHB * 4; ++ks) {
-#pragma unroll
-            for (int k = 0; k < HPW; ++k) {
-              if (sw + kSoftmaxWarps * k >= H_own) continue;
-              uint32_t a[4];
-              ldmatrix_x4(kt + a_off[k][rb][ks], a);
-              mma_16816_bf16(acc[k], a, bq[k][ks][0], bq[k][ks][1]);
+            for (int j = 0; j < DH / 8; ++j) {
+              const int colk = hh * DH + 8 * j;
+              uint4 kv;
+              asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(kv.x), "=r"(kv.y), "=r"(kv.z), "=r"(kv.w)
+                           : "r"(rbase + (colk >> 6) * 2048 + ((((colk & 63) >> 3) ^ (row & 7)) << 4)));
+              const float4 qa = qv[2 * j], qb = qv[2 * j + 1];
+              a0 = fmaf(bf16lo(kv.x), qa.x, a0);
+              a1 = fmaf(bf16hi(kv.x), qa.y, a1);
+              a0 = fmaf(bf16lo(kv.y), qa.z, a0);
+              a1 = fmaf(bf16hi(kv.y), qa.w, a1);
+              a0 = fmaf(bf16lo(kv.z), qb.x, a0);
+              a1 = fmaf(bf16hi(kv.z), qb.y, a1);
+              a0 = fmaf(bf16lo(kv.w), qb.z, a0);
+              a1 = fmaf(bf16hi(kv.w), qb.w, a1);
             }
           }
-#pragma unroll
-          for (int k = 0; k < HPW; ++k) {
-            sc[k][2 * rb] = acc[k][0] + acc[k][1];
-            sc[k][2 * rb + 1] = acc[k][2] + acc[k][3];
-          }
+          sc[ps] = (k < HPW && hh < H_own && row < nvalid) ? (a0 + a1) * p.scale_log2 : -INFINITY;
         }
-        // Phase 2: tile maxima of every head, shuffle trees interleaved
-        float mx[HPW];
+        // Phase 2: tile maxima (over the TT lanes of a head)
+        float mx[NPASS];
 #pragma unroll
-        for (int k = 0; k < HPW; ++k) {
-          mx[k] = -INFINITY;
+        for (int ps = 0; ps < NPASS; ++ps) mx[ps] = sc[ps];
 #pragma unroll
-          for (int i = 0; i < TT / 8; ++i) {
-            const int trow = 8 * i + gq;  // (rb, half) = (i / 2, i % 2): row 16 rb + 8 half + gq
-            sc[k][i] = (tq == 0 && trow < nvalid) ? sc[k][i] * p.scale_log2 : -INFINITY;
-            mx[k] = fmaxf(mx[k], sc[k][i]);
-          }
-        }
+        for (int o = TT / 2; o > 0; o >>= 1)
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-          for (int k = 0; k < HPW; ++k) mx[k] = fmaxf(mx[k], __shfl_xor_sync(0xffffffffu, mx[k], o));
+          for (int ps = 0; ps < NPASS; ++ps) mx[ps] = fmaxf(mx[ps], __shfl_xor_sync(0xffffffffu, mx[ps], o));
         // Phase 3: lazy running max, P to shared memory (and the cluster peers)
 #pragma unroll
-        for (int k = 0; k < HPW; ++k) {
+        for (int ps = 0; ps < NPASS; ++ps) {
+          const int k = ps * HPP + hslot;
           const int hh = sw + kSoftmaxWarps * k;
-          if (hh >= H_own) continue;
+          if (k >= HPW || hh >= H_own) continue;
           float alpha = 1.f;
           if (t == 0) {
-            mref[k] = mx[k];
-          } else if (mx[k] > mref[k] + kLazyRescaleLog2) {
-            alpha = exp2f(mref[k] - mx[k]);
-            mref[k] = mx[k];
-            lsum[k] *= alpha;
+            mref[ps] = mx[ps];
+          } else if (mx[ps] > mref[ps] + kLazyRescaleLog2) {
+            alpha = exp2f(mref[ps] - mx[ps]);
+            mref[ps] = mx[ps];
+            lsum[ps] *= alpha;
           }
           const int n = head0 + hh;
           const int m = p_row(n);
-          if (tq == 0) {
+          const float pv = row < nvalid ? exp2f(sc[ps] - mref[ps]) : 0.f;
+          const __nv_bfloat16 pb = __float2bfloat16_rn(pv);
+          lsum[ps] += __bfloat162float(pb);
+          const uint32_t off = static_cast<uint32_t>(s) * pstage_bytes +
+                               static_cast<uint32_t>(((m >> 3) * (TT / 8) + (row >> 3)) * 128 + (m & 7) * 16 + (row & 7) * 2);
+          const uint16_t bits = __bfloat16_as_ushort(pb);
+          asm volatile("st.shared.u16 [%0], %1;" ::"r"(pst_base + off), "h"(bits) : "memory");
 #pragma unroll
-            for (int i = 0; i < TT / 8; ++i) {
-              const int trow = 8 * i + gq;
-              const float pv = (trow < nvalid) ? exp2f(sc[k][i] - mref[k]) : 0.f;
-              const __nv_bfloat16 pb = __float2bfloat16_rn(pv);
-              lsum[k] += __bfloat162float(pb);
-              const uint32_t off = static_cast<uint32_t>(s) * pstage_bytes +
-                                   static_cast<uint32_t>(((m >> 3) * (TT / 8) + i) * 128 + (m & 7) * 16 + gq * 2);
-              const uint16_t bits = __bfloat16_as_ushort(pb);
-              asm volatile("st.shared.u16 [%0], %1;" ::"r"(pst_base + off), "h"(bits) : "memory");
-#pragma unroll
-              for (int r = 1; r < CL; ++r) st_cluster_u16(mapa_shared(pst_base + off, (rank + r) % CL), bits);
-            }
-          }
-          if (lane == 0) {
+          for (int r = 1; r < CL; ++r) st_cluster_u16(mapa_shared(pst_base + off, (rank + r) % CL), bits);
+          if (row == 0) {
             alpha_s[s * kPRows + n] = alpha;
 #pragma unroll
             for (int r = 1; r < CL; ++r)
@@ -522,11 +494,14 @@ __global__ void __launch_bounds__(kTCThreads, 1)
       if (!ok) break;
       const size_t slot = static_cast<size_t>(item);
 #pragma unroll
-      for (int k = 0; k < HPW; ++k) {
+      for (int ps = 0; ps < NPASS; ++ps) {
+        const int k = ps * HPP + hslot;
         const int hh = sw + kSoftmaxWarps * k;
-        const float tot = warp_sum(lsum[k]);
-        if (hh < H_own && lane == 0) {
-          p.ws_m[slot * p.H + head0 + hh] = mref[k];
+        float tot = lsum[ps];
+#pragma unroll
+        for (int o = TT / 2; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+        if (k < HPW && hh < H_own && row == 0) {
+          p.ws_m[slot * p.H + head0 + hh] = mref[ps];
           p.ws_l[slot * p.H + head0 + hh] = tot;
         }
       }
@@ -534,6 +509,9 @@ __global__ void __launch_bounds__(kTCThreads, 1)
   }
 
   // ---------------------------------------------------------------- teardown
+  // Reconverge every warp first: in the producer and MMA warps only lane 0 ran
+  // the loop, and a CTA barrier reached by a split warp does not wait for it.
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -605,8 +583,30 @@ bool pick_config(int B, int d, int H, TCConfig* out) {
   return false;
 }
 
+// Clusters of CL CTAs that can be resident at once. A cluster must fit in one
+// GPC, so with CL > 1 fewer than num_sms / CL clusters may fit; launching more
+// would run the extra ones as a second wave. Memoised per (device, smem).
 template <int CL, int TT, int DHB, int HPW>
-cudaError_t launch_tc(const CUtensorMap& map, const DecodeTCParams& prm, const TCConfig& c, cudaStream_t st) {
+int resident_clusters(cudaLaunchConfig_t cfg) {
+  static std::mutex mu;
+  static std::map<std::pair<int, uint32_t>, int> memo;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  const std::pair<int, uint32_t> key(dev, static_cast<uint32_t>(cfg.dynamicSmemBytes));
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = memo.find(key);
+  if (it != memo.end()) return it->second;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, decode_b_tc_kernel<CL, TT, DHB, HPW>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  memo[key] = n;
+  return n;
+}
+
+template <int CL, int TT, int DHB, int HPW>
+cudaError_t launch_tc(const CUtensorMap& map, DecodeTCParams prm, const TCConfig& c, cudaStream_t st) {
   auto kern = decode_b_tc_kernel<CL, TT, DHB, HPW>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(c.smem));
   if (e != cudaSuccess) return e;
@@ -616,14 +616,25 @@ cudaError_t launch_tc(const CUtensorMap& map, const DecodeTCParams& prm, const T
   cfg.dynamicSmemBytes = c.smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  attr[1].id = cudaLaunchAttributeClusterDimension;
-  attr[1].val.clusterDim.x = CL;
-  attr[1].val.clusterDim.y = 1;
-  attr[1].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = CL > 1 ? 2 : 1;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  if (CL > 1) {
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const int fit = resident_clusters<CL, TT, DHB, HPW>(cfg);
+    if (fit > 0 && fit < prm.n_groups) {
+      prm.n_groups = fit;
+      cfg.gridDim = dim3(static_cast<unsigned>(fit * CL), 1, 1);
+    }
+    cfg.numAttrs = 2;
+  } else {
+    cfg.attrs = attr + 1;
+    cfg.numAttrs = 1;
+  }
   return cudaLaunchKernelEx(&cfg, kern, map, prm);
 }
 

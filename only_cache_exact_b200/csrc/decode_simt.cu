@@ -86,8 +86,8 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(const SimtParams p) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (warp == 0)
-    plan_split(p.lens, p.B, p.cap, p.attend_add, p.n_slots, p.n_slots, p.min_rows, s_nb, s_rows, s_off, p.ws_meta, p.status,
-               blockIdx.x == 0);
+    plan_split(p.lens, p.B, p.cap, p.attend_add, p.n_slots, p.n_slots, p.min_rows, s_nb, s_rows, s_off, p.ws_meta,
+               p.status, blockIdx.x == 0);
   __syncthreads();
   const SplitItem it = plan_lookup(blockIdx.x, p.B, s_nb, s_rows, s_off);
   if (it.b < 0) return;

@@ -150,6 +150,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
   }
+  __syncwarp();  // lanes 1..31 of warps 0 and 1 skipped the lane-0 loops: reconverge before the CTA barrier
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

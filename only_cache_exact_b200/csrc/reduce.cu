@@ -6,12 +6,21 @@
 // rule into  ū = Σ_c 2^(m_c - M) U_c / Σ_c 2^(m_c - M) l_c,  M = max_c m_c,
 // and the head output is  o[b, h-cols] = ū · W_KV[:, h-cols].
 //
-// Grid (H, NDB) with clusters of NDB CTAs along y: CTA (h, r) merges the
-// d-block r of ū for every sequence and multiplies it by the matching
-// d-block rows of W_KV's head-h columns; the NDB partial products are summed
-// through distributed shared memory (deterministic order) and written once.
-// The kernel is launched as a programmatic dependent of the split kernel: it
-// prefetches its W_KV block into L2 before waiting for the partials.
+// The merge is small and latency-bound, so it is laid out to wait for memory
+// as few times as possible. Grid (H, NDB), clusters of NDB CTAs along y; CTA
+// (h, r) owns head h and the d-block r (DB = d / NDB columns).
+//   * Before the split kernel's results are awaited, its W_KV block (DB rows of
+//     the head-h columns; a parameter, not a result) is requested by TMA.
+//   * Then every thread issues all its loads at once: its items' slice of U
+//     (16-byte loads, two rounds of eight in flight), and the items' m and l.
+//   * One warp per sequence turns m, l into merge weights; each thread scales
+//     its U rows and adds them, per sequence, into ū in shared memory.
+//   * o_r[b, :] = ū[b, block] · W_KV[block, h-cols] on mma.sync (bf16 W_KV; ū
+//     as a bf16 high + low pair, fp32 accumulation) or fp32 FMAs (fp32 W_KV).
+//   * Each CTA pushes its product into the owner CTA of every output element
+//     (distributed shared memory) and signals the owner's mbarrier; owners add
+//     the NDB products in a fixed order and write o.
+// The kernel is a programmatic dependent of the split kernel.
 //
 // Ordering (a) needs only the merge (its partials are already softmax·V).
 #include <cuda_bf16.h>
@@ -22,208 +31,290 @@
 
 namespace slim {
 
-struct ReduceBParams {
+struct MergeBParams {
   const float* U;
   const float* m;
   const float* l;
   const int32_t* meta;
-  const void* w_kv;
   float* out;
   int32_t* lens;
   int32_t* status;
   int B, d, H, ndb, max_items;
-  int sb;           // sequences per cluster reduction round
+  int b_begin, nb;  // sequences of this launch
+  int use_mma;      // bf16 W_KV, d_h a multiple of 64: swizzled W block, tensor-core projection
+  int cap_ranges;   // the split fills (nearly) every work slot: item runs sized by the capacity
 };
 
-constexpr int kReduceThreads = 256;
-constexpr int kReduceNBB = 8;  // sequences per projection block (register accumulators)
+constexpr int kMergeThreads = 256;
+constexpr int kMergeWarps = kMergeThreads / 32;
+constexpr int kMergeMaxSeqs = 128;  // sequences per launch (MMA rows)
+constexpr int kMergeMaxTiles = 8;   // 16x8 output tiles per warp
+constexpr int kMergeRound = 8;      // 16-byte loads in flight per thread and round
 
-template <typename WT>
-struct WVec;
-template <>
-struct WVec<__nv_bfloat16> {
-  static constexpr int N = 8;
-  __device__ __forceinline__ static void load(const __nv_bfloat16* p, float (&w)[8]) {
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
-    w[0] = bf16lo(v.x); w[1] = bf16hi(v.x); w[2] = bf16lo(v.y); w[3] = bf16hi(v.y);
-    w[4] = bf16lo(v.z); w[5] = bf16hi(v.z); w[6] = bf16lo(v.w); w[7] = bf16hi(v.w);
-  }
+struct MergeSmem {
+  uint32_t w, ub, ubs, wts, ls, soff, part, recv, per, bars, total;
 };
-template <>
-struct WVec<float> {
-  static constexpr int N = 4;
-  __device__ __forceinline__ static void load(const float* p, float (&w)[4]) {
-    const float4 v = __ldg(reinterpret_cast<const float4*>(p));
-    w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
-  }
-};
-
-struct ReduceSmem {
-  uint32_t wts, ubar, part, red, total;
-};
-__host__ __device__ inline ReduceSmem reduce_smem_layout(int max_items, int DB, int d_h, int sb) {
-  ReduceSmem r;
+__host__ __device__ inline uint32_t up_to(uint32_t x, uint32_t a) { return (x + a - 1u) / a * a; }
+__host__ __device__ inline MergeSmem merge_smem_layout(int DB, int d_h, int esz, int nb, int ndb, int ncap) {
+  MergeSmem s;
   uint32_t o = 0;
-  r.wts = o;
-  o += ((static_cast<uint32_t>(max_items) + 3u) & ~3u) * 4u;
-  r.ubar = o;
-  o += static_cast<uint32_t>(kReduceNBB) * DB * 4u;
-  r.part = o;
-  o += static_cast<uint32_t>(sb) * d_h * 4u;
-  r.red = o;
-  o += static_cast<uint32_t>(kReduceThreads / 32) * kReduceNBB * d_h * 4u;
-  r.total = o;
-  return r;
+  s.w = o;  // W_KV block [DB rows][d_h]: 64-column 128-byte-swizzled boxes (MMA) or dense rows
+  o += up_to(static_cast<uint32_t>(DB) * d_h * esz, 1024u);
+  s.ubs = static_cast<uint32_t>(DB) + 8u;  // row stride of ū (floats), padded against bank conflicts
+  s.ub = o;
+  o += up_to(static_cast<uint32_t>(nb), 16u) * s.ubs * 4u;
+  s.wts = o;
+  o += up_to(static_cast<uint32_t>(ncap), 4u) * 4u;
+  s.ls = o;
+  o += up_to(static_cast<uint32_t>(ncap), 4u) * 4u;
+  s.soff = o;
+  o += up_to(static_cast<uint32_t>(nb) + 1u, 4u) * 4u;
+  s.part = o;  // this CTA's product [nb][d_h]
+  o += static_cast<uint32_t>(nb) * d_h * 4u;
+  s.per = (static_cast<uint32_t>(nb) * d_h + ndb - 1u) / ndb;  // output elements owned per CTA
+  s.recv = o;  // products pushed by the NDB CTAs of the cluster: [NDB][per]
+  o += static_cast<uint32_t>(ndb) * s.per * 4u;
+  o = up_to(o, 8u);
+  s.bars = o;
+  o += 16u;
+  s.total = o + 1024u;  // slack to align the base to 1024 bytes
+  return s;
 }
 
 template <typename WT>
-__global__ void __launch_bounds__(kReduceThreads) reduce_b_kernel(const ReduceBParams p) {
-  extern __shared__ __align__(16) uint8_t rsm[];
-  constexpr int VEC = WVec<WT>::N;
+__global__ void __launch_bounds__(kMergeThreads, 2)
+    merge_b_kernel(const __grid_constant__ CUtensorMap wmap, const MergeBParams p) {
+  extern __shared__ uint8_t msm_raw[];
+  uint8_t* msm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(msm_raw) + 1023) & ~uintptr_t(1023));
   const int h = blockIdx.x, r = blockIdx.y;
-  const int d_h = p.d / p.H;
-  const int DB = p.d / p.ndb, c0 = r * DB;
+  const int d_h = p.d / p.H, DB = p.d / p.ndb, c0 = r * DB;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const WT* W = static_cast<const WT*>(p.w_kv);
-  const ReduceSmem L = reduce_smem_layout(p.max_items, DB, d_h, p.sb);
-  float* wts = reinterpret_cast<float*>(rsm + L.wts);
-  float* ubar = reinterpret_cast<float*>(rsm + L.ubar);
-  float* part = reinterpret_cast<float*>(rsm + L.part);
-  float* red = reinterpret_cast<float*>(rsm + L.red);
+  const int nb = p.nb, b0 = p.b_begin, Bp = (nb + 15) & ~15;
+  const MergeSmem L = merge_smem_layout(DB, d_h, static_cast<int>(sizeof(WT)), nb, p.ndb, p.max_items);
+  float* ub = reinterpret_cast<float*>(msm + L.ub);
+  float* wts = reinterpret_cast<float*>(msm + L.wts);  // m of every item, then its merge weight
+  float* ls = reinterpret_cast<float*>(msm + L.ls);
+  int* s_off = reinterpret_cast<int*>(msm + L.soff);  // items of sequence b0 + i start at s_off[i]
+  float* part = reinterpret_cast<float*>(msm + L.part);
+  float* recv = reinterpret_cast<float*>(msm + L.recv);
+  uint64_t* wbar = reinterpret_cast<uint64_t*>(msm + L.bars);
+  const int ubs = static_cast<int>(L.ubs), per = static_cast<int>(L.per);
 
-  // Before the partials exist: pull this CTA's W_KV block (rows c0.., head-h columns) into L2.
-  {
-    const int row_bytes = d_h * static_cast<int>(sizeof(WT));
-    const int lines = (row_bytes + 127) / 128;
-    for (int i = tid; i < DB * lines; i += kReduceThreads) {
-      const int row = i / lines, ln = i % lines;
-      const char* a = reinterpret_cast<const char*>(W + static_cast<size_t>(c0 + row) * p.d + h * d_h) + ln * 128;
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
-    }
+  // ---- before the split kernel's results exist: barrier, W_KV block, zeroed ū
+  if (tid == 0) {
+    mbar_init(wbar, 1);
+    fence_barrier_init();
+    tma_prefetch_desc(&wmap);
+    const int groups = p.use_mma ? d_h / 64 : 1, gcols = p.use_mma ? 64 : d_h, yrows = min(DB, 256);
+    mbar_arrive_expect_tx(wbar, static_cast<uint32_t>(DB) * d_h * sizeof(WT));
+    for (int g = 0; g < groups; ++g)
+      for (int y = 0; y < DB; y += yrows)
+        tma_load_2d(msm + L.w + static_cast<size_t>(g * DB + y) * gcols * sizeof(WT), &wmap, h * d_h + g * 64, c0 + y,
+                    wbar, l2_policy_evict_last());
   }
+  for (int i = tid; i < Bp * ubs; i += kMergeThreads) ub[i] = 0.f;
+  if (p.ndb > 1) cluster_arrive_relaxed();
   pdl_wait_primary();
   pdl_launch_dependents();
+
+  // ---- every load at once: this thread's U slices, then the work list and m, l
+  const int it0 = b0 == 0 ? 0 : __ldcg(p.meta + 1 + b0);
+  const int ncap = p.max_items - it0;
+  // Thread (cg, ig) takes columns 4cg.. of a contiguous run of items (runs of one sequence
+  // then add up in registers). When the split fills nearly every work slot the runs are sized
+  // by the capacity, so the first loads need no read of the work list; otherwise they are
+  // balanced over the items the split kernel produced.
+  const int C4 = DB / 4, IG = kMergeThreads / C4;
+  const int cg = tid % C4, ig = tid < IG * C4 ? tid / C4 : IG;
+  int ipt = (ncap + IG - 1) / IG, n_real = ncap;
+  if (!p.cap_ranges) {
+    n_real = min(ncap, __ldcg(p.meta + 1 + b0 + nb) - it0);  // items of this launch's sequences
+    ipt = (n_real + IG - 1) / IG;
+  }
+  const int i_beg = ig * ipt;
+  int i_end = ig < IG ? min(n_real, i_beg + ipt) : i_beg;
+  const float4* ubase = reinterpret_cast<const float4*>(p.U + (static_cast<size_t>(it0) * p.H + h) * p.d + c0) + cg;
+  const size_t istride = static_cast<size_t>(p.H) * p.d / 4;  // float4 stride between items
+  const int nrounds = (ipt + kMergeRound - 1) / kMergeRound;
+  float4 bufA[kMergeRound], bufB[kMergeRound];
+  auto load_round = [&](float4 (&buf)[kMergeRound], int rr) {
+#pragma unroll
+    for (int u = 0; u < kMergeRound; ++u) {
+      const int i = i_beg + rr * kMergeRound + u;
+      buf[u] = i < i_end ? __ldcg(ubase + static_cast<size_t>(i) * istride) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  load_round(bufA, 0);
+  if (p.cap_ranges) i_end = min(i_end, __ldcg(p.meta + 1 + b0 + nb) - it0);  // later rounds: real items only
+  if (nrounds > 1) load_round(bufB, 1);
+  for (int i = tid; i <= nb; i += kMergeThreads) s_off[i] = __ldcg(p.meta + 1 + b0 + i) - it0;
+  for (int i = tid; i < ncap; i += kMergeThreads) {
+    wts[i] = __ldcg(p.m + static_cast<size_t>(it0 + i) * p.H + h);
+    ls[i] = __ldcg(p.l + static_cast<size_t>(it0 + i) * p.H + h);
+  }
+  if (h == 0 && r == 0)
+    for (int b = b0 + tid; b < b0 + nb; b += kMergeThreads)
+      if (__ldcg(p.meta + 2 + p.B + b) & kSeqAppend) p.lens[b] += 1;
   __syncthreads();
 
-  const int32_t* off = p.meta + 1;
-  if (h == 0 && r == 0) {
-    for (int b = tid; b < p.B; b += kReduceThreads)
-      if (p.meta[2 + p.B + b] & kSeqAppend) p.lens[b] += 1;
-  }
-
-  // merge weights 2^(m_c - M) / L of every item c for head h
-  for (int b = warp; b < p.B; b += kReduceThreads / 32) {
-    const int c_lo = off[b], c_hi = off[b + 1];
+  // ---- merge weights 2^(m_c - M) / Σ_c' 2^(m_c' - M) l_c', one warp per sequence
+  for (int bl = warp; bl < nb; bl += kMergeWarps) {
+    const int lo = s_off[bl], hi = s_off[bl + 1];
     float M = -INFINITY;
-    for (int c = c_lo + lane; c < c_hi; c += 32) M = fmaxf(M, p.m[static_cast<size_t>(c) * p.H + h]);
+    for (int c = lo + lane; c < hi; c += 32) M = fmaxf(M, wts[c]);
     M = warp_max(M);
-    float Ls = 0.f;
-    for (int c = c_lo + lane; c < c_hi; c += 32)
-      Ls += exp2f(p.m[static_cast<size_t>(c) * p.H + h] - M) * p.l[static_cast<size_t>(c) * p.H + h];
-    Ls = warp_sum(Ls);
-    const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
-    for (int c = c_lo + lane; c < c_hi; c += 32) wts[c] = exp2f(p.m[static_cast<size_t>(c) * p.H + h] - M) * inv;
+    float S = 0.f;
+    for (int c = lo + lane; c < hi; c += 32) S += exp2f(wts[c] - M) * ls[c];
+    S = warp_sum(S);
+    const float inv = S > 0.f ? 1.f / S : 0.f;
+    for (int c = lo + lane; c < hi; c += 32) wts[c] = exp2f(wts[c] - M) * inv;
   }
   __syncthreads();
 
-  const int ncg = d_h / VEC;               // column groups of VEC columns
-  const int G = kReduceThreads / ncg;      // row groups
-  const int cg = tid % ncg, g = tid / ncg;
-  const int gpw = 32 / ncg;                // row groups per warp (ncg <= 32)
-  const uint32_t part_base = smem_u32(part);
+  // ---- ū[b, block] = Σ_c w_c U_c[block]: runs of one sequence add up in registers
+  if (i_beg < i_end) {
+    int bcur = 0;
+    while (bcur < nb && s_off[bcur + 1] <= i_beg) ++bcur;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    auto flush = [&]() {
+      if (bcur < nb) {
+        float* dst = ub + bcur * ubs + 4 * cg;
+        red_shared_add(dst, acc.x);
+        red_shared_add(dst + 1, acc.y);
+        red_shared_add(dst + 2, acc.z);
+        red_shared_add(dst + 3, acc.w);
+      }
+      acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    };
+    auto consume = [&](const float4 (&buf)[kMergeRound], int rr) {
+#pragma unroll
+      for (int u = 0; u < kMergeRound; ++u) {
+        const int i = i_beg + rr * kMergeRound + u;
+        if (i >= i_end) break;
+        while (bcur < nb && i >= s_off[bcur + 1]) {
+          flush();
+          ++bcur;
+        }
+        if (bcur >= nb) break;
+        const float w = wts[i];
+        acc.x = fmaf(w, buf[u].x, acc.x);
+        acc.y = fmaf(w, buf[u].y, acc.y);
+        acc.z = fmaf(w, buf[u].z, acc.z);
+        acc.w = fmaf(w, buf[u].w, acc.w);
+      }
+    };
+    for (int rr = 0; rr < nrounds; rr += 2) {
+      consume(bufA, rr);
+      if (rr + 2 < nrounds) load_round(bufA, rr + 2);
+      if (rr + 1 < nrounds) {
+        consume(bufB, rr + 1);
+        if (rr + 3 < nrounds) load_round(bufB, rr + 3);
+      }
+    }
+    flush();
+  }
+  const bool ok = __syncthreads_and(mbar_wait(wbar, 0u, p.status));
 
-  for (int s0 = 0; s0 < p.B; s0 += p.sb) {
-    const int nsb = min(p.sb, p.B - s0);
-    for (int b0 = s0; b0 < s0 + nsb; b0 += kReduceNBB) {
-      const int nbb = min(kReduceNBB, s0 + nsb - b0);
-      // ū of the block straight from the partials: float4 loads, eight items in flight per thread
-      const int nv = DB / 4;
-      const size_t item4 = static_cast<size_t>(p.H) * p.d / 4;  // float4 stride between items
-      for (int i = tid; i < kReduceNBB * nv; i += kReduceThreads) {
-        const int bl = i / nv, c4 = i % nv;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (bl < nbb) {
-          const int lo = off[b0 + bl], hi = off[b0 + bl + 1];
-          const float4* src =
-              reinterpret_cast<const float4*>(p.U + (static_cast<size_t>(lo) * p.H + h) * p.d + c0) + c4;
-          int c = lo;
-          for (; c + 8 <= hi; c += 8) {
-            float4 v[8];
+  // ---- this CTA's product o_r[b, :] = ū[b, block] · W_KV[block, h-cols]
+  if (ok && p.use_mma && nb > 4) {
+    // 16x8 tiles: rows = sequences, columns = 8 of the head's d_h; ū = hi + lo in bf16
+    const int NT = d_h / 8, T = (Bp / 16) * NT;
+    const uint32_t wbase = smem_u32(msm + L.w);
+    const int g = lane >> 2, tq = lane & 3;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) v[u] = __ldg(src + u * item4);
+    for (int i = 0; i < kMergeMaxTiles; ++i) {
+      const int t = warp + kMergeWarps * i;
+      if (t >= T) break;
+      const int mt = t / NT, nt = t - mt * NT;
+      const int wb = nt >> 3, chunk = nt & 7;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int ks = 0; ks < DB / 16; ++ks) {
+        const int row = ks * 16 + (lane & 15);
+        uint32_t b0f, b1f;
+        ldmatrix_x2_trans(wbase + (wb * DB + row) * 128 + ((chunk ^ (row & 7)) << 4), b0f, b1f);
+        const float* a = ub + (mt * 16 + g) * ubs + ks * 16 + 2 * tq;
+        const float2 xs[4] = {*reinterpret_cast<const float2*>(a), *reinterpret_cast<const float2*>(a + 8 * ubs),
+                              *reinterpret_cast<const float2*>(a + 8), *reinterpret_cast<const float2*>(a + 8 * ubs + 8)};
+        uint32_t ahi[4], alo[4];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const float w = wts[c + u];
-              acc.x = fmaf(w, v[u].x, acc.x);
-              acc.y = fmaf(w, v[u].y, acc.y);
-              acc.z = fmaf(w, v[u].z, acc.z);
-              acc.w = fmaf(w, v[u].w, acc.w);
-            }
-            src += 8 * item4;
-          }
-          for (; c < hi; ++c, src += item4) {
-            const float4 v = __ldg(src);
-            const float w = wts[c];
-            acc.x = fmaf(w, v.x, acc.x);
-            acc.y = fmaf(w, v.y, acc.y);
-            acc.z = fmaf(w, v.z, acc.z);
-            acc.w = fmaf(w, v.w, acc.w);
-          }
+        for (int e = 0; e < 4; ++e) {
+          const __nv_bfloat16 h0 = __float2bfloat16_rn(xs[e].x), h1 = __float2bfloat16_rn(xs[e].y);
+          ahi[e] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
+                   (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+          alo[e] = pack_bf16x2(xs[e].x - __bfloat162float(h0), xs[e].y - __bfloat162float(h1));
         }
-        *reinterpret_cast<float4*>(ubar + bl * DB + 4 * c4) = acc;
+        mma_16816_bf16(acc, ahi, b0f, b1f);
+        mma_16816_bf16(acc, alo, b0f, b1f);
       }
-      __syncthreads();
-      // partial head output of the block: ū[bl, d-block] · W_KV[d-block rows, head-h columns]
-      float acc[kReduceNBB][VEC];
+      const int row = mt * 16 + g, col = nt * 8 + 2 * tq;
+      if (row < nb) *reinterpret_cast<float2*>(part + row * d_h + col) = make_float2(acc[0], acc[1]);
+      if (row + 8 < nb) *reinterpret_cast<float2*>(part + (row + 8) * d_h + col) = make_float2(acc[2], acc[3]);
+    }
+  } else if (ok) {
+    // FMAs: thread -> (sequence, 4 columns, one of S interleaved row subsets of the block),
+    // the S partial sums (adjacent lanes) added with shuffles
+    const WT* wsm = reinterpret_cast<const WT*>(msm + L.w);
+    const int pairs = nb * (d_h / 4);
+    int S = 1;
+    while (S < 32 && pairs * S * 2 <= kMergeThreads) S *= 2;
+    for (int q0 = 0; q0 < pairs * S; q0 += kMergeThreads) {
+      const int q = q0 + tid;
+      const int pr = q / S, cs = q % S;
+      const int bl = pr / (d_h / 4), j = 4 * (pr - bl * (d_h / 4));
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (pr < pairs) {
+        for (int c = cs; c < DB; c += S) {
+          const float u = ub[bl * ubs + c];
+          float w[4];
+          if (p.use_mma) {  // swizzled 64-column boxes of bf16
+            const int wb = j >> 6, jj = j & 63;
+            const uint8_t* rowp = msm + L.w + static_cast<size_t>(wb * DB + c) * 128;
+            const uint2 v = *reinterpret_cast<const uint2*>(rowp + ((((jj >> 3) ^ (c & 7)) << 4) | ((jj & 7) * 2)));
+            w[0] = bf16lo(v.x);
+            w[1] = bf16hi(v.x);
+            w[2] = bf16lo(v.y);
+            w[3] = bf16hi(v.y);
+          } else {
+            const WT* wr = wsm + static_cast<size_t>(c) * d_h + j;
 #pragma unroll
-      for (int bl = 0; bl < kReduceNBB; ++bl)
-#pragma unroll
-        for (int v = 0; v < VEC; ++v) acc[bl][v] = 0.f;
-      if (g < G) {
-        const WT* wp = W + static_cast<size_t>(c0) * p.d + h * d_h + cg * VEC;
-#pragma unroll 4
-        for (int i = g; i < DB; i += G) {
-          float w[VEC];
-          WVec<WT>::load(wp + static_cast<size_t>(i) * p.d, w);
-#pragma unroll
-          for (int bl = 0; bl < kReduceNBB; ++bl) {
-            const float u = ubar[bl * DB + i];
-#pragma unroll
-            for (int v = 0; v < VEC; ++v) acc[bl][v] = fmaf(u, w[v], acc[bl][v]);
+            for (int v = 0; v < 4; ++v) w[v] = static_cast<float>(wr[v]);
           }
+          a.x = fmaf(u, w[0], a.x);
+          a.y = fmaf(u, w[1], a.y);
+          a.z = fmaf(u, w[2], a.z);
+          a.w = fmaf(u, w[3], a.w);
         }
       }
-      // reduce the row groups of a warp with shuffles, then across warps through shared memory
-#pragma unroll
-      for (int bl = 0; bl < kReduceNBB; ++bl)
-#pragma unroll
-        for (int v = 0; v < VEC; ++v)
-          for (int o = ncg; o < 32; o <<= 1) acc[bl][v] += __shfl_xor_sync(0xffffffffu, acc[bl][v], o);
-      if (lane < ncg && g < G) {
-#pragma unroll
-        for (int bl = 0; bl < kReduceNBB; ++bl)
-#pragma unroll
-          for (int v = 0; v < VEC; ++v) red[(warp * kReduceNBB + bl) * d_h + cg * VEC + v] = acc[bl][v];
+      for (int o = 1; o < S; o <<= 1) {
+        a.x += __shfl_xor_sync(0xffffffffu, a.x, o);
+        a.y += __shfl_xor_sync(0xffffffffu, a.y, o);
+        a.z += __shfl_xor_sync(0xffffffffu, a.z, o);
+        a.w += __shfl_xor_sync(0xffffffffu, a.w, o);
       }
-      __syncthreads();
-      const int nwarps = min(kReduceThreads / 32, (G + gpw - 1) / gpw);
-      for (int i = tid; i < nbb * d_h; i += kReduceThreads) {
-        float sum = 0.f;
-        for (int w2 = 0; w2 < nwarps; ++w2) sum += red[w2 * kReduceNBB * d_h + i];
-        part[(b0 - s0) * d_h + i] = sum;
-      }
-      __syncthreads();
+      if (pr < pairs && cs == 0) *reinterpret_cast<float4*>(part + bl * d_h + j) = a;
     }
-    // sum the NDB CTAs' products through distributed shared memory (fixed order)
-    cluster_sync();
-    for (int i = tid; i < nsb * d_h; i += kReduceThreads) {
-      if (i % p.ndb != r) continue;
-      float sum = 0.f;
-      for (int q = 0; q < p.ndb; ++q) sum += ld_cluster_f32(mapa_shared(part_base + 4u * i, q));
-      const int bl = i / d_h, jj = i % d_h;
-      p.out[static_cast<size_t>(s0 + bl) * p.d + h * d_h + jj] = sum;
-    }
-    cluster_sync();
+  }
+  __syncthreads();
+
+  // ---- sum the NDB products: push each element to its owner CTA, then add in a fixed order
+  const int n_out = nb * d_h;
+  if (p.ndb == 1) {
+    for (int e = tid; e < n_out; e += kMergeThreads)
+      p.out[static_cast<size_t>(b0 + e / d_h) * p.d + h * d_h + e % d_h] = ok ? part[e] : 0.f;
+    return;
+  }
+  cluster_wait();  // every CTA of the cluster is running
+  const uint32_t recv_base = smem_u32(recv);
+  for (int e = tid; e < n_out; e += kMergeThreads)
+    st_cluster_f32(mapa_shared(recv_base + 4u * static_cast<uint32_t>(r * per + e / p.ndb), e % p.ndb),
+                   ok ? part[e] : 0.f);
+  cluster_sync();  // pushes visible; nobody touches a peer's shared memory after this
+  for (int s = tid; s < per; s += kMergeThreads) {
+    const int e = s * p.ndb + r;
+    if (e >= n_out) break;
+    float a = 0.f;
+    for (int q = 0; q < p.ndb; ++q) a += recv[q * per + s];
+    p.out[static_cast<size_t>(b0 + e / d_h) * p.d + h * d_h + e % d_h] = a;
   }
 }
 
@@ -263,59 +354,109 @@ __global__ void __launch_bounds__(256) reduce_a_kernel(const ReduceAParams p) {
 
 // ---------------------------------------------------------------------------- host
 namespace {
-int pick_ndb(int d, int d_h) {
-  // d-blocks per head: a cluster of up to 8 CTAs; blocks stay multiples of 8 columns.
-  for (int n = 8; n >= 1; --n)
-    if (d % n == 0 && (d / n) % 8 == 0) return n;
-  return 1;
+
+struct MergeConfig {
+  int ndb, use_mma, nb_max;
+  size_t smem;
+};
+
+// NDB: the smallest of 1, 2, 4, 8 that gives at least one CTA per SM, preferring a
+// footprint that lets two CTAs share an SM; 16 (a non-portable cluster) only when no
+// smaller block fits.
+bool pick_merge(int B, int d, int H, int esz, int max_items, MergeConfig* c) {
+  const int d_h = d / H;
+  const bool mma = esz == 2 && d_h % 64 == 0;
+  if (!mma && (d_h % 4 || (d_h * esz) % 16 || d_h > 256)) return false;
+  c->use_mma = mma ? 1 : 0;
+  c->nb_max = mma ? std::min(kMergeMaxSeqs, 16 * kMergeWarps * kMergeMaxTiles / (d_h / 8)) : kMergeMaxSeqs;
+  const int nb = std::min(B, c->nb_max);
+  const size_t half = static_cast<size_t>(max_smem_optin()) / 2 - 2048, full = static_cast<size_t>(max_smem_optin()) - 2048;
+  // rank 3: enough CTAs and two per SM; 2: enough CTAs; 1: fits (the most blocks wins)
+  int best = 0, best_rank = 0;
+  size_t best_smem = 0;
+  for (int ndb = 1; ndb <= 16; ndb *= 2) {
+    if (ndb == 16 && best != 0) break;
+    if (d % ndb) break;
+    const int DB = d / ndb;
+    if (DB % (mma ? 16 : 4) || (DB > 256 && DB % 256) || DB / 4 > kMergeThreads) continue;
+    const size_t sm = merge_smem_layout(DB, d_h, esz, nb, ndb, max_items).total;
+    if (sm > full) continue;
+    const bool enough = H * ndb >= num_sms();
+    const int rank = enough ? (sm <= half ? 3 : 2) : 1;
+    if (rank > best_rank || (rank == 1 && best_rank == 1)) {
+      best = ndb;
+      best_rank = rank;
+      best_smem = sm;
+    }
+    if (rank == 3) break;
+  }
+  if (best == 0) return false;
+  c->ndb = best;
+  c->smem = best_smem;
+  return true;
 }
+
 }  // namespace
 
 cudaError_t launch_reduce_b(const DecodeArgs& a, const SplitWorkspace& ws, bool pdl, cudaStream_t st,
                             int* launches) {
+  const int esz = a.dtype == SLIM_BF16 ? 2 : 4;
   const int d_h = a.d / a.H;
-  const int vec = (a.dtype == SLIM_BF16) ? 8 : 4;
-  if (d_h % vec || d_h / vec > 32 || (32 % (d_h / vec)) != 0) return cudaErrorNotSupported;
-  ReduceBParams p;
-  p.U = ws.U;
-  p.m = ws.m;
-  p.l = ws.l;
-  p.meta = ws.meta;
-  p.w_kv = a.w_kv;
-  p.out = a.out;
-  p.lens = a.lens;
-  p.status = a.status;
-  p.B = a.B;
-  p.d = a.d;
-  p.H = a.H;
-  p.ndb = pick_ndb(a.d, d_h);
-  p.max_items = ws.max_items;
-  const int DB = a.d / p.ndb;
-  if (DB % 4) return cudaErrorNotSupported;
-  p.sb = std::max(kReduceNBB, std::min(a.B, (32 * 1024) / (d_h * 4)) / kReduceNBB * kReduceNBB);
-  p.sb = std::min(p.sb, ((a.B + kReduceNBB - 1) / kReduceNBB) * kReduceNBB);
-  const size_t smem = reduce_smem_layout(p.max_items, DB, d_h, p.sb).total;
-  if (smem > 200u * 1024u) return cudaErrorNotSupported;
-  auto kern = (a.dtype == SLIM_BF16) ? reduce_b_kernel<__nv_bfloat16> : reduce_b_kernel<float>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  MergeConfig c;
+  if (!pick_merge(a.B, a.d, a.H, esz, ws.max_items, &c)) return cudaErrorNotSupported;
+  const int DB = a.d / c.ndb;
+  // W_KV as {d columns, d rows}; a box is one 64-column swizzled group (MMA) or the head's d_h columns
+  CUtensorMap wmap;
+  const uint64_t dims[2] = {static_cast<uint64_t>(a.d), static_cast<uint64_t>(a.d)};
+  const uint64_t strides[1] = {static_cast<uint64_t>(a.d) * esz};
+  const uint32_t box[2] = {static_cast<uint32_t>(c.use_mma ? 64 : d_h), static_cast<uint32_t>(std::min(DB, 256))};
+  if (!encode_tmap(&wmap, esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, a.w_kv,
+                   dims, strides, box, c.use_mma != 0))
+    return cudaErrorInvalidValue;
+  // The tcgen05 split with single-CTA groups (CL = 1) plans one item per SM slot, so its
+  // items nearly fill the workspace capacity; other configurations leave most slots empty.
+  const bool cap_ranges = a.dtype == SLIM_BF16 && decode_b_tc_cluster(a.B, a.d, a.H) == 1;
+  auto kern = (a.dtype == SLIM_BF16) ? merge_b_kernel<__nv_bfloat16> : merge_b_kernel<float>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(c.smem));
+  if (e == cudaSuccess && c.ndb > 8) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(a.H), static_cast<unsigned>(p.ndb), 1);
-  cfg.blockDim = dim3(kReduceThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = static_cast<unsigned>(p.ndb);
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  e = cudaLaunchKernelEx(&cfg, kern, p);
-  if (e == cudaSuccess && launches) ++*launches;
-  return e;
+  for (int b0 = 0; b0 < a.B; b0 += c.nb_max) {
+    MergeBParams p;
+    p.U = ws.U;
+    p.m = ws.m;
+    p.l = ws.l;
+    p.meta = ws.meta;
+    p.out = a.out;
+    p.lens = a.lens;
+    p.status = a.status;
+    p.B = a.B;
+    p.d = a.d;
+    p.H = a.H;
+    p.ndb = c.ndb;
+    p.max_items = ws.max_items;
+    p.b_begin = b0;
+    p.nb = std::min(c.nb_max, a.B - b0);
+    p.use_mma = c.use_mma;
+    p.cap_ranges = cap_ranges ? 1 : 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(a.H), static_cast<unsigned>(c.ndb), 1);
+    cfg.blockDim = dim3(kMergeThreads, 1, 1);
+    cfg.dynamicSmemBytes = merge_smem_layout(DB, d_h, esz, p.nb, c.ndb, ws.max_items).total;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = static_cast<unsigned>(c.ndb);
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = (pdl && b0 == 0) ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    e = cudaLaunchKernelEx(&cfg, kern, wmap, p);
+    if (e != cudaSuccess) return e;
+    if (launches) ++*launches;
+  }
+  return cudaSuccess;
 }
 
 cudaError_t launch_reduce_a(const DecodeArgs& a, const SplitWorkspace& ws, cudaStream_t st, int* launches) {

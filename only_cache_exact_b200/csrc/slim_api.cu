@@ -84,6 +84,24 @@ bool encode_tmap_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64
   return r == CUDA_SUCCESS;
 }
 
+bool encode_tmap(CUtensorMap* map, CUtensorMapDataType type, int rank, const void* base, const uint64_t* dims,
+                 const uint64_t* strides, const uint32_t* box, bool swizzle128) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn || rank < 1 || rank > 5) return false;
+  cuuint64_t dd[5], ss[4];
+  cuuint32_t bb[5], ee[5];
+  for (int i = 0; i < rank; ++i) {
+    dd[i] = dims[i];
+    bb[i] = box[i];
+    ee[i] = 1;
+    if (i + 1 < rank) ss[i] = strides[i];
+  }
+  CUresult r = fn(map, type, static_cast<cuuint32_t>(rank), const_cast<void*>(base), dd, ss, bb, ee,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool encode_tmap_kslab(CUtensorMap* map, const void* base, uint64_t rows, int d, int box_blocks) {
   if (d % 64 || box_blocks < 1 || box_blocks > 256) return false;
   return encode_tmap_3d_bf16(map, base, 64, rows, static_cast<uint64_t>(d / 64), static_cast<uint64_t>(d) * 2u, 128,

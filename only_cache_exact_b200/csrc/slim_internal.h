@@ -54,6 +54,8 @@ struct SplitPlan {
 // Variant (b), tcgen05 path (bf16). Returns cudaErrorNotSupported if the shape has no tcgen05 config.
 cudaError_t launch_decode_b_tc(const DecodeArgs& a, const SplitWorkspace& ws, cudaStream_t st, int* launches);
 bool decode_b_tc_supported(int B, int d, int H);
+// Cluster size of the tcgen05 split kernel for this shape (0: no tcgen05 configuration).
+int decode_b_tc_cluster(int B, int d, int H);
 // Variant (b), CUDA-core path (fp32 or bf16 cache).
 cudaError_t launch_decode_b_simt(const DecodeArgs& a, const SplitWorkspace& ws, cudaStream_t st, int* launches);
 bool decode_b_simt_supported(int B, int d, int H);
@@ -83,6 +85,10 @@ bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uin
 // dims 1 and 2, box {b0, b1, b2}, 128-byte swizzle (b0 * 2 must be <= 128).
 bool encode_tmap_3d_bf16(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
                          uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2);
+// Tiled map of any rank <= 5: dims (innermost first), byte strides of dims 1.., box; no
+// interleave, optional 128-byte swizzle, zero fill out of range.
+bool encode_tmap(CUtensorMap* map, CUtensorMapDataType type, int rank, const void* base, const uint64_t* dims,
+                 const uint64_t* strides, const uint32_t* box, bool swizzle128);
 // K cache [rows][d] bf16 as a 3-D map {64 columns, rows, d/64 column blocks} with a box of
 // 64 x 16 x box_blocks, 128-byte swizzle: one load brings 16 rows of box_blocks column blocks.
 bool encode_tmap_kslab(CUtensorMap* map, const void* base, uint64_t rows, int d, int box_blocks);

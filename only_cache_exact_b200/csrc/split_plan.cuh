@@ -9,17 +9,6 @@
 
 namespace slim {
 
-__device__ __forceinline__ long long warp_sum_ll(long long v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-__device__ __forceinline__ int warp_sum_int(int v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
 struct SplitItem {
   int b;     // sequence, -1 if this slot has no work
   int row0;  // first row of the chunk within the sequence
@@ -50,7 +39,7 @@ __device__ inline int plan_chunk(const int* s_nb, int B, long long n_slots, int 
     const int C = mid << 4;
     int cnt = 0;
     for (int b = lane; b < B; b += 32) cnt += (s_nb[b] + C - 1) / C;
-    cnt = warp_sum_int(cnt);
+    cnt = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(cnt)));
     if (cnt <= n_slots) hi = mid; else lo = mid + 1;
   }
   return lo << 4;
@@ -70,7 +59,7 @@ __device__ inline void plan_split(const int32_t* __restrict__ lens, int B, int64
   int bad = 0, nonempty = 0, max_nb = 0;
   long long R = 0;
   for (int b = lane; b < B; b += 32) {
-    const int L = __ldg(lens + b);
+    const int L = __ldcg(lens + b);
     int nb;
     if (L < 0 || static_cast<int64_t>(L) > cap) {
       nb = 0;
@@ -87,8 +76,9 @@ __device__ inline void plan_split(const int32_t* __restrict__ lens, int B, int64
     max_nb = max(max_nb, nb);
     if (report) meta[2 + B + b] = (nb > 0 && append) ? kSeqAppend : 0;
   }
-  R = warp_sum_ll(R);
-  nonempty = warp_sum_int(nonempty);
+  // attended rows fit in 31 bits (B * cap < 2^31), so single-instruction warp reductions suffice
+  R = static_cast<long long>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(R)));
+  nonempty = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(nonempty)));
   max_nb = __reduce_max_sync(0xffffffffu, max_nb);
   bad = __reduce_or_sync(0xffffffffu, bad);
   if (report && lane == 0 && bad) atomicOr(status, bad);
@@ -103,7 +93,7 @@ __device__ inline void plan_split(const int32_t* __restrict__ lens, int B, int64
     const int C = plan_chunk(s_nb, B, n_slots, min_rows, R, nonempty, max_nb);
     int items = 0;
     for (int b = lane; b < B; b += 32) items += (s_nb[b] + C - 1) / C;
-    items = warp_sum_int(items);
+    items = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(items)));
     const long long per_group = (items + n_groups - 1) / n_groups;
     const long long est = per_group * (C + kItemCostRows);
     if (best < 0 || est < best) {
