@@ -236,3 +236,29 @@ def test_ordering_a_d4096(S):
     c = make_case(4096, 32, lens=[200, 37], cap=300, seed=12)
     g = GpuState(c, S)
     _check_bf16(g.step(S.SLIM_VARIANT_A), oracle_out(c), c.H)
+
+
+def test_selector_tunes_then_auto_step_matches(S):
+    """slim_tune measures both orderings at several T, restores lens, and SLIM_AUTO then runs the
+    recorded winner; the step it runs still matches the oracle."""
+    c = make_case(1024, 16, lens=[900, 900], cap=1200, append=False, seed=11)
+    g = GpuState(c, S)
+    dt = S.SLIM_BF16
+    S.slim_tune_clear()
+    assert S.slim_select_variant(dt, c.B, c.d, c.H, 900) == S.SLIM_VARIANT_B  # empty table: (b)
+    Ts = [16, 128, 900]
+    S.slim_tune(g.q, g.K, g.lens, torch.from_numpy(c.lens), g.W_KV, c.H, Ts, 3, g.out, g.ws, g.status)
+    torch.cuda.synchronize()
+    assert torch.equal(g.lens.cpu(), torch.from_numpy(c.lens))  # restored
+    assert int(g.status.item()) == 0
+    picks = [S.slim_select_variant(dt, c.B, c.d, c.H, t) for t in Ts]
+    assert all(v in (S.SLIM_VARIANT_A, S.SLIM_VARIANT_B) for v in picks)
+    # ordering (a) materialises V = K·W_KV (a d x d GEMM per row): at T = 900 it cannot win
+    assert picks[-1] == S.SLIM_VARIANT_B
+    # a recorded point where (a) is faster flips the choice near that T only
+    S.slim_tune_record(dt, c.B, c.d, c.H, 16, 0.001, 1.0)
+    assert S.slim_select_variant(dt, c.B, c.d, c.H, 16) == S.SLIM_VARIANT_A
+    assert S.slim_select_variant(dt, c.B, c.d, c.H, 900) == S.SLIM_VARIANT_B
+    got = g.step(S.SLIM_AUTO)
+    _check_bf16(got, oracle_out(c), c.H)
+    S.slim_tune_clear()
