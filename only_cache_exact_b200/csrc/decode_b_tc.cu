@@ -22,8 +22,9 @@
 //                TMEM (lane offsets 0 and 16), so 1024 columns fit in the 512
 //                TMEM columns.
 //   warps 2..5   correction and epilogue: the lazy online-softmax rescale of
-//                the accumulator rows whose max grew by more than 2^8, and
-//                TMEM -> partials in global memory.
+//                the accumulator rows whose max grew by more than 2^8 (the MMA
+//                warp waits for this pass only on tiles a score warp flagged),
+//                and TMEM -> partials in global memory.
 //   warps 6..13  scores: per head, q_h·K_t on the CUDA cores, one K row per
 //                lane (16-byte loads from the swizzled stage, q broadcast from
 //                shared memory, fp32 accumulation), running max, P in bf16 to
@@ -74,7 +75,7 @@ struct DecodeTCParams {
 
 // Shared-memory carve-up, identical on host and device.
 struct TCSmem {
-  uint32_t k_off, p_off, alpha_off, q_off, bar_off, slot_off, plan_off, total;
+  uint32_t k_off, p_off, alpha_off, flag_off, q_off, bar_off, slot_off, plan_off, total;
 };
 __host__ __device__ inline TCSmem tc_smem_layout(int CL, int TT, int d, int stages, int B) {
   TCSmem s;
@@ -86,6 +87,8 @@ __host__ __device__ inline TCSmem tc_smem_layout(int CL, int TT, int d, int stag
   o += static_cast<uint32_t>(stages) * kPRows * TT * 2u;
   s.alpha_off = o;
   o += static_cast<uint32_t>(stages) * kPRows * 4u;
+  s.flag_off = o;  // per stage: the tile index whose heads need a rescale (else older)
+  o += static_cast<uint32_t>(stages) * 4u;
   o = (o + 15u) & ~15u;
   s.q_off = o;
   o += dS * 4u;
@@ -121,6 +124,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
   uint8_t* kst = smem + L.k_off;
   uint8_t* pst = smem + L.p_off;
   float* alpha_s = reinterpret_cast<float*>(smem + L.alpha_off);
+  volatile int* resc = reinterpret_cast<volatile int*>(smem + L.flag_off);
   float* q_s = reinterpret_cast<float*>(smem + L.q_off);  // this CTA's columns of q
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar_off);
   uint64_t* full = bars;                       // TMA landed (tx bytes)
@@ -166,6 +170,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
     uint32_t* pz = reinterpret_cast<uint32_t*>(pst);
     for (uint32_t i = t; i < stages * pstage_bytes / 4u; i += kSoftmaxWarps * 32) pz[i] = 0u;
     for (int i = t; i < stages * kPRows; i += kSoftmaxWarps * 32) alpha_s[i] = 1.0f;
+    for (int i = t; i < stages; i += kSoftmaxWarps * 32) resc[i] = -1;
     fence_proxy_async_smem();
   }
   pdl_wait_primary();
@@ -225,7 +230,10 @@ __global__ void __launch_bounds__(kTCThreads, 1)
         for (int t = 0; t < nt; ++t, ++g) {
           const int s = g % stages;
           const uint32_t ph = static_cast<uint32_t>(g / stages) & 1u;
-          if (!mbar_wait(&corr[s], ph, p.status) || !mbar_wait(&full[s], ph, p.status)) {
+          // P of every head written (this CTA and its peers) and the K stage landed; the
+          // correction warps' pass is awaited only for a tile in which some head rescales
+          if (!mbar_wait<(CL > 1)>(&pfull[s], ph, p.status) || !mbar_wait(&full[s], ph, p.status) ||
+              (resc[s] == g && !mbar_wait(&corr[s], ph, p.status))) {
             ok = false;
             break;
           }
@@ -400,8 +408,10 @@ __global__ void __launch_bounds__(kTCThreads, 1)
           __syncwarp();
         }
 
-        // P stage s is free once the MMAs that read it (tile g - stages) finished in every CTA.
-        if (g >= stages && !__all_sync(0xffffffffu, mbar_wait<(CL > 1)>(&pempty[s], ph ^ 1u, p.status))) {
+        // P stage s is free once the MMAs that read it (tile g - stages) finished in every CTA
+        // and this CTA's correction warps have read its alphas.
+        if (g >= stages && !__all_sync(0xffffffffu, mbar_wait<(CL > 1)>(&pempty[s], ph ^ 1u, p.status) &&
+                                                        mbar_wait(&corr[s], ph ^ 1u, p.status))) {
           ok = false;
           break;
         }
@@ -450,6 +460,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
 #pragma unroll
           for (int ps = 0; ps < NPASS; ++ps) mx[ps] = fmaxf(mx[ps], __shfl_xor_sync(0xffffffffu, mx[ps], o));
         // Phase 3: lazy running max, P to shared memory (and the cluster peers)
+        bool rescaled = false;
 #pragma unroll
         for (int ps = 0; ps < NPASS; ++ps) {
           const int k = ps * HPP + hslot;
@@ -462,6 +473,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
             alpha = exp2f(mref[ps] - mx[ps]);
             mref[ps] = mx[ps];
             lsum[ps] *= alpha;
+            rescaled = true;
           }
           const int n = head0 + hh;
           const int m = p_row(n);
@@ -481,6 +493,12 @@ __global__ void __launch_bounds__(kTCThreads, 1)
               st_cluster_f32(mapa_shared(alpha_base + static_cast<uint32_t>((s * kPRows + n) * 4), (rank + r) % CL),
                              alpha);
           }
+        }
+        if (__any_sync(0xffffffffu, rescaled) && lane == 0) {
+          resc[s] = g;
+#pragma unroll
+          for (int r = 1; r < CL; ++r)
+            st_cluster_f32(mapa_shared(smem_u32(const_cast<int*>(resc + s)), (rank + r) % CL), __int_as_float(g));
         }
         fence_proxy_async_smem();
         if (CL > 1) fence_proxy_async_cluster();
