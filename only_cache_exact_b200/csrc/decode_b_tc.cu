@@ -25,9 +25,11 @@
 //                the accumulator rows whose max grew by more than 2^8 (the MMA
 //                warp waits for this pass only on tiles a score warp flagged),
 //                and TMEM -> partials in global memory.
-//   warps 6..13  scores: per head, q_h·K_t on the CUDA cores, one K row per
-//                lane (16-byte loads from the swizzled stage, q broadcast from
-//                shared memory, fp32 accumulation), running max, P in bf16 to
+//   warps 6..13  scores: per head, q_h·K_t on the CUDA cores (32-row tiles: a
+//                lane multiplies one 16-byte chunk of 8 rows by q held in
+//                registers, a butterfly over the 8 chunk lanes sums the rows;
+//                16-row tiles: one row per lane, q broadcast from shared
+//                memory), fp32 accumulation, running max, P in bf16 to
 //                shared memory and to the other CTAs of the cluster
 //                (distributed shared memory). The tensor pipe is left to the
 //                P·K MMAs.
@@ -337,7 +339,10 @@ __global__ void __launch_bounds__(kTCThreads, 1)
     const int sw = warp - 6;  // heads sw, sw + 8, ... of this CTA
     constexpr int HPP = 32 / TT;                  // heads per pass (one row per lane)
     constexpr int NPASS = (HPW + HPP - 1) / HPP;  // passes over this warp's heads
-    const int row = lane % TT, hslot = lane / TT;
+    // TT = 32: lane (chunk c = lane % 8, row group rg = lane / 8) multiplies 16-byte chunk c of
+    // rows rg, rg + 4, ... by q held in registers, and a butterfly over the 8 chunk lanes leaves
+    // row rg + 4 c in the lane. TT = 16: one row per lane, two heads per pass.
+    const int row = TT == 32 ? (lane >> 3) + 4 * (lane & 7) : lane % TT, hslot = lane / TT;
     const uint32_t kbase = smem_u32(kst);
     const uint32_t pst_base = smem_u32(pst);
     const uint32_t alpha_base = smem_u32(alpha_s);
@@ -348,8 +353,10 @@ __global__ void __launch_bounds__(kTCThreads, 1)
       const int nt = tiles_of(it);
       const int b = it.b;
       const int nb_old = it.nb - p.append;  // rows holding cached keys
-      // q of this warp's heads to shared memory (read back as broadcasts)
+      // q of this warp's heads to shared memory (read back as broadcasts, or kept in registers
+      // for this lane's chunks when TT = 32)
       float mref[NPASS], lsum[NPASS];  // running max and sum of this lane's head in each pass
+      float qr[TT == 32 ? HPW : 1][DHB][8];
 #pragma unroll
       for (int ps = 0; ps < NPASS; ++ps) {
         mref[ps] = -INFINITY;
@@ -366,6 +373,19 @@ __global__ void __launch_bounds__(kTCThreads, 1)
         }
       }
       __syncwarp();
+      if constexpr (TT == 32) {
+#pragma unroll
+        for (int k = 0; k < HPW; ++k) {
+          const int hh = sw + kSoftmaxWarps * k;
+#pragma unroll
+          for (int jj = 0; jj < DHB; ++jj) {
+            const float4* qv = reinterpret_cast<const float4*>(q_s + (hh < H_own ? hh : 0) * DH + 8 * ((lane & 7) + 8 * jj));
+            const float4 qa = qv[0], qb = qv[1];
+            qr[k][jj][0] = qa.x; qr[k][jj][1] = qa.y; qr[k][jj][2] = qa.z; qr[k][jj][3] = qa.w;
+            qr[k][jj][4] = qb.x; qr[k][jj][5] = qb.y; qr[k][jj][6] = qb.z; qr[k][jj][7] = qb.w;
+          }
+        }
+      }
 
       for (int t = 0; t < nt; ++t, ++g) {
         const int s = g % stages;
@@ -417,39 +437,90 @@ __global__ void __launch_bounds__(kTCThreads, 1)
         }
 
         const uint32_t kt = kbase + s * kstage_bytes;
-        // Phase 1: scores on the CUDA cores (the tensor pipe is left to the P·K MMAs).
-        // Lane -> (row, head slot): row = lane % TT, and with TT = 16 the two half-warps
-        // take alternate heads. A lane reads its row's d_h columns of the head once
-        // (16-byte loads from the swizzled stage, conflict-free), q as broadcasts, and
-        // accumulates in fp32.
+        // Phase 1: scores on the CUDA cores (the tensor pipe is left to the P·K MMAs), fp32
+        // accumulation, K read once from the swizzled stage with conflict-free 16-byte loads.
         float sc[NPASS];
+        if constexpr (TT == 32) {
+          const int c = lane & 7, rg = lane >> 3;
 #pragma unroll
-        for (int ps = 0; ps < NPASS; ++ps) {
-          const int k = ps * HPP + hslot;
-          const int hh = sw + kSoftmaxWarps * k;
-          float a0 = 0.f, a1 = 0.f;
-          if (k < HPW && hh < H_own) {
-            const uint32_t rbase = kt + (row >> 4) * slab_bytes + (row & 15) * 128;
-            const float4* qv = reinterpret_cast<const float4*>(q_s + hh * DH);
+          for (int k = 0; k < HPW; ++k) {
+            const int hh = sw + kSoftmaxWarps * k;
+            sc[k] = -INFINITY;
+            if (hh >= H_own) continue;  // warp-uniform: this warp has no head in slot k
+            float pr[8];
 #pragma unroll
-            for (int j = 0; j < DH / 8; ++j) {
-              const int colk = hh * DH + 8 * j;
-              uint4 kv;
-              asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                           : "=r"(kv.x), "=r"(kv.y), "=r"(kv.z), "=r"(kv.w)
-                           : "r"(rbase + (colk >> 6) * 2048 + ((((colk & 63) >> 3) ^ (row & 7)) << 4)));
-              const float4 qa = qv[2 * j], qb = qv[2 * j + 1];
-              a0 = fmaf(bf16lo(kv.x), qa.x, a0);
-              a1 = fmaf(bf16hi(kv.x), qa.y, a1);
-              a0 = fmaf(bf16lo(kv.y), qa.z, a0);
-              a1 = fmaf(bf16hi(kv.y), qa.w, a1);
-              a0 = fmaf(bf16lo(kv.z), qb.x, a0);
-              a1 = fmaf(bf16hi(kv.z), qb.y, a1);
-              a0 = fmaf(bf16lo(kv.w), qb.z, a0);
-              a1 = fmaf(bf16hi(kv.w), qb.w, a1);
+            for (int i = 0; i < 8; ++i) {
+              const int r = rg + 4 * i;
+              const uint32_t rbase = kt + (r >> 4) * slab_bytes + (r & 15) * 128;
+              float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+              for (int jj = 0; jj < DHB; ++jj) {
+                const int colk = hh * DH + 8 * (c + 8 * jj);
+                uint4 kv;
+                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(kv.x), "=r"(kv.y), "=r"(kv.z), "=r"(kv.w)
+                             : "r"(rbase + (colk >> 6) * 2048 + ((((colk & 63) >> 3) ^ (r & 7)) << 4)));
+                a0 = fmaf(bf16lo(kv.x), qr[k][jj][0], a0);
+                a1 = fmaf(bf16hi(kv.x), qr[k][jj][1], a1);
+                a0 = fmaf(bf16lo(kv.y), qr[k][jj][2], a0);
+                a1 = fmaf(bf16hi(kv.y), qr[k][jj][3], a1);
+                a0 = fmaf(bf16lo(kv.z), qr[k][jj][4], a0);
+                a1 = fmaf(bf16hi(kv.z), qr[k][jj][5], a1);
+                a0 = fmaf(bf16lo(kv.w), qr[k][jj][6], a0);
+                a1 = fmaf(bf16hi(kv.w), qr[k][jj][7], a1);
+              }
+              pr[i] = a0 + a1;
             }
+            // butterfly over the chunk lanes: after the level with mask m each lane keeps the
+            // rows whose index bit (m) matches its own chunk bit, summed over both lanes
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const bool up = c & 4;
+              const float recv = __shfl_xor_sync(0xffffffffu, up ? pr[i] : pr[i + 4], 4);
+              pr[i] = (up ? pr[i + 4] : pr[i]) + recv;
+            }
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const bool up = c & 2;
+              const float recv = __shfl_xor_sync(0xffffffffu, up ? pr[i] : pr[i + 2], 2);
+              pr[i] = (up ? pr[i + 2] : pr[i]) + recv;
+            }
+            {
+              const bool up = c & 1;
+              const float recv = __shfl_xor_sync(0xffffffffu, up ? pr[0] : pr[1], 1);
+              pr[0] = (up ? pr[1] : pr[0]) + recv;
+            }
+            sc[k] = row < nvalid ? pr[0] * p.scale_log2 : -INFINITY;
           }
-          sc[ps] = (k < HPW && hh < H_own && row < nvalid) ? (a0 + a1) * p.scale_log2 : -INFINITY;
+        } else {
+#pragma unroll
+          for (int ps = 0; ps < NPASS; ++ps) {
+            const int k = ps * HPP + hslot;
+            const int hh = sw + kSoftmaxWarps * k;
+            float a0 = 0.f, a1 = 0.f;
+            if (k < HPW && hh < H_own) {
+              const uint32_t rbase = kt + (row >> 4) * slab_bytes + (row & 15) * 128;
+              const float4* qv = reinterpret_cast<const float4*>(q_s + hh * DH);
+#pragma unroll
+              for (int j = 0; j < DH / 8; ++j) {
+                const int colk = hh * DH + 8 * j;
+                uint4 kv;
+                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(kv.x), "=r"(kv.y), "=r"(kv.z), "=r"(kv.w)
+                             : "r"(rbase + (colk >> 6) * 2048 + ((((colk & 63) >> 3) ^ (row & 7)) << 4)));
+                const float4 qa = qv[2 * j], qb = qv[2 * j + 1];
+                a0 = fmaf(bf16lo(kv.x), qa.x, a0);
+                a1 = fmaf(bf16hi(kv.x), qa.y, a1);
+                a0 = fmaf(bf16lo(kv.y), qa.z, a0);
+                a1 = fmaf(bf16hi(kv.y), qa.w, a1);
+                a0 = fmaf(bf16lo(kv.z), qb.x, a0);
+                a1 = fmaf(bf16hi(kv.z), qb.y, a1);
+                a0 = fmaf(bf16lo(kv.w), qb.z, a0);
+                a1 = fmaf(bf16hi(kv.w), qb.w, a1);
+              }
+            }
+            sc[ps] = (k < HPW && hh < H_own && row < nvalid) ? (a0 + a1) * p.scale_log2 : -INFINITY;
+          }
         }
         // Phase 2: tile maxima (over the TT lanes of a head)
         float mx[NPASS];

@@ -126,15 +126,6 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* map, int32_t 
 }
 
 // ------------------------------------------------------------------ cluster
-// 1-D bulk copy global -> this CTA's shared memory, completing on `bar` (no
-// multicast). Both addresses and `bytes` must be multiples of 16.
-__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   smem_u32(dst)),
-               "l"(src), "r"(bytes), "r"(smem_u32(bar))
-               : "memory");
-}
-
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
