@@ -21,16 +21,18 @@ struct SplitItem {
 // items. Bracketed first: C >= R / n_slots is necessary, and
 // C >= R / (n_slots - nonempty) is sufficient (ceil adds at most one chunk per
 // sequence), so the binary search usually runs a handful of steps. One warp.
-__device__ inline int plan_chunk(const int* s_nb, int B, long long n_slots, int min_rows, long long R, int nonempty,
+// All quantities fit in 32 bits (R = attended rows < 2^31): the divisions stay
+// 32-bit, which keeps this dependent chain short.
+__device__ inline int plan_chunk(const int* s_nb, int B, unsigned n_slots, int min_rows, unsigned R, int nonempty,
                                  int max_nb) {
   const int lane = threadIdx.x & 31;
   const int cap16 = max((max_nb + 15) >> 4, 1);
   int lo = (max(min_rows, 16) + 15) >> 4;
-  lo = max(lo, static_cast<int>((R + n_slots * 16 - 1) / (n_slots * 16)));
+  lo = max(lo, static_cast<int>((R + 16u * n_slots - 1u) / (16u * n_slots)));  // ceil(R / (16 n_slots))
   int hi = cap16;
-  if (n_slots > nonempty) {
-    const long long free_slots = n_slots - nonempty;
-    hi = min(hi, static_cast<int>((R + free_slots * 16 - 1) / (free_slots * 16)));
+  if (n_slots > static_cast<unsigned>(nonempty)) {
+    const unsigned free_slots = n_slots - static_cast<unsigned>(nonempty);
+    hi = min(hi, static_cast<int>((R + 16u * free_slots - 1u) / (16u * free_slots)));
   }
   if (lo >= hi) return max(lo, 1) << 4;
 #pragma unroll 1
@@ -38,9 +40,9 @@ __device__ inline int plan_chunk(const int* s_nb, int B, long long n_slots, int 
     const int mid = (lo + hi) >> 1;
     const int C = mid << 4;
     int cnt = 0;
-    for (int b = lane; b < B; b += 32) cnt += (s_nb[b] + C - 1) / C;
+    for (int b = lane; b < B; b += 32) cnt += static_cast<int>((static_cast<unsigned>(s_nb[b]) + C - 1) / C);
     cnt = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(cnt)));
-    if (cnt <= n_slots) hi = mid; else lo = mid + 1;
+    if (static_cast<unsigned>(cnt) <= n_slots) hi = mid; else lo = mid + 1;
   }
   return lo << 4;
 }
@@ -88,13 +90,13 @@ __device__ inline void plan_split(const int32_t* __restrict__ lens, int B, int64
   int chunk = 16;
   long long best = -1;
   for (int k = 1; static_cast<long long>(k) * n_groups <= max_items || k == 1; k <<= 1) {
-    const long long n_slots = max(static_cast<long long>(k) * n_groups, static_cast<long long>(nonempty));
-    if (n_slots > max_items && k > 1) break;
-    const int C = plan_chunk(s_nb, B, n_slots, min_rows, R, nonempty, max_nb);
+    const unsigned n_slots = static_cast<unsigned>(max(k * n_groups, nonempty));
+    if (n_slots > static_cast<unsigned>(max_items) && k > 1) break;
+    const int C = plan_chunk(s_nb, B, n_slots, min_rows, static_cast<unsigned>(R), nonempty, max_nb);
     int items = 0;
-    for (int b = lane; b < B; b += 32) items += (s_nb[b] + C - 1) / C;
+    for (int b = lane; b < B; b += 32) items += static_cast<int>((static_cast<unsigned>(s_nb[b]) + C - 1) / C);
     items = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(items)));
-    const long long per_group = (items + n_groups - 1) / n_groups;
+    const long long per_group = static_cast<long long>((static_cast<unsigned>(items) + n_groups - 1) / n_groups);
     const long long est = per_group * (C + kItemCostRows);
     if (best < 0 || est < best) {
       best = est;
@@ -110,7 +112,7 @@ __device__ inline void plan_split(const int32_t* __restrict__ lens, int B, int64
     if (b < B) {
       const int nb = s_nb[b];
       s_rows[b] = chunk;
-      if (nb > 0) c = (nb + chunk - 1) / chunk;
+      if (nb > 0) c = static_cast<int>((static_cast<unsigned>(nb) + chunk - 1) / chunk);
     }
     int x = c;
 #pragma unroll
