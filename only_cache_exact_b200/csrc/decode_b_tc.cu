@@ -20,19 +20,21 @@
 //                N <= 256 (columns), K = 16 rows; the K slab is read in place
 //                as the MN-major B operand. Two M=64 accumulators interleave in
 //                TMEM (lane offsets 0 and 16), so 1024 columns fit in the 512
-//                TMEM columns.
+//                TMEM columns. With CL > 1 it first sends this CTA's rows of
+//                P and alpha to every peer as one bulk shared-to-shared copy
+//                each (completing on the peer's mbarrier): one hop through
+//                distributed shared memory per tile, no cluster-scope fence.
 //   warps 2..5   correction and epilogue: the lazy online-softmax rescale of
 //                the accumulator rows whose max grew by more than 2^8 (the MMA
-//                warp waits for this pass only on tiles a score warp flagged),
-//                and TMEM -> partials in global memory.
+//                warp waits for this pass first only on tiles with a rescaled
+//                row), and TMEM -> partials in global memory.
 //   warps 6..13  scores: per head, q_h·K_t on the CUDA cores (32-row tiles: a
 //                lane multiplies one 16-byte chunk of 8 rows by q held in
 //                registers, a butterfly over the 8 chunk lanes sums the rows;
 //                16-row tiles: one row per lane, q broadcast from shared
-//                memory), fp32 accumulation, running max, P in bf16 to
-//                shared memory and to the other CTAs of the cluster
-//                (distributed shared memory). The tensor pipe is left to the
-//                P·K MMAs.
+//                memory), fp32 accumulation, running max, P in bf16 and the
+//                rescale factors to this CTA's rows of the stage. The tensor
+//                pipe is left to the P·K MMAs.
 // Every mbarrier wait is bounded; a timeout sets SLIM_DEV_TIMEOUT and the
 // kernel drains its copies and MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
@@ -77,7 +79,7 @@ struct DecodeTCParams {
 
 // Shared-memory carve-up, identical on host and device.
 struct TCSmem {
-  uint32_t k_off, p_off, alpha_off, flag_off, q_off, bar_off, slot_off, plan_off, total;
+  uint32_t k_off, p_off, alpha_off, q_off, bar_off, slot_off, plan_off, total;
 };
 __host__ __device__ inline TCSmem tc_smem_layout(int CL, int TT, int d, int stages, int B) {
   TCSmem s;
@@ -87,16 +89,13 @@ __host__ __device__ inline TCSmem tc_smem_layout(int CL, int TT, int d, int stag
   o += static_cast<uint32_t>(stages) * TT * dS * 2u;
   s.p_off = o;
   o += static_cast<uint32_t>(stages) * kPRows * TT * 2u;
-  s.alpha_off = o;
+  s.alpha_off = o;  // per stage: the rescale factor of every P row (1 = none)
   o += static_cast<uint32_t>(stages) * kPRows * 4u;
-  s.flag_off = o;  // per stage: the tile index whose heads need a rescale (else older)
-  o += static_cast<uint32_t>(stages) * 4u;
-  o = (o + 15u) & ~15u;
   s.q_off = o;
   o += dS * 4u;
   o = (o + 7u) & ~7u;
   s.bar_off = o;
-  o += (5u * stages + 2u) * 8u;
+  o += (6u * stages + 2u) * 8u;
   s.slot_off = o;
   o += 16u;
   s.plan_off = o;
@@ -105,9 +104,21 @@ __host__ __device__ inline TCSmem tc_smem_layout(int CL, int TT, int d, int stag
   return s;
 }
 
-// Row of head n in the P operand / accumulator: heads n, n+4, ... share the
-// TMEM lane quarter n % 4, so the correction warps split the rows evenly.
-__host__ __device__ inline int p_row(int n) { return 16 * (n & 3) + (n >> 2); }
+// Row of head n in the P operand and the accumulator. CTA r of a cluster owns
+// heads [r·H_own, (r+1)·H_own) and the contiguous rows [r·64/CL, (r+1)·64/CL),
+// so its part of P (and of alpha) is one block it can copy to its peers. The
+// 16-row TMEM lane quarters of that block take its heads in turn (j, j + 4/CL,
+// ... share a quarter), so the four correction warps split the rows evenly.
+__host__ __device__ inline int p_row(int n, int CL, int H_own) {
+  const int qpr = 4 / CL, r = n / H_own, j = n - r * H_own;
+  return r * (kPRows / CL) + 16 * (j % qpr) + j / qpr;
+}
+// The inverse: the head in row i, or -1 for a padding row.
+__host__ __device__ inline int row_head(int i, int CL, int H_own) {
+  const int R = kPRows / CL, qpr = 4 / CL, r = i / R, w = i - r * R;
+  const int j = (w % 16) * qpr + w / 16;
+  return j < H_own ? r * H_own + j : -1;
+}
 
 template <int CL, int TT, int DHB, int HPW>
 __global__ void __launch_bounds__(kTCThreads, 1)
@@ -125,17 +136,17 @@ __global__ void __launch_bounds__(kTCThreads, 1)
   const TCSmem L = tc_smem_layout(CL, TT, p.d, stages, p.B);
   uint8_t* kst = smem + L.k_off;
   uint8_t* pst = smem + L.p_off;
-  float* alpha_s = reinterpret_cast<float*>(smem + L.alpha_off);
-  volatile int* resc = reinterpret_cast<volatile int*>(smem + L.flag_off);
+  float* alpha_s = reinterpret_cast<float*>(smem + L.alpha_off);  // [stages][kPRows], by P row
   float* q_s = reinterpret_cast<float*>(smem + L.q_off);  // this CTA's columns of q
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar_off);
   uint64_t* full = bars;                       // TMA landed (tx bytes)
   uint64_t* empty = bars + stages;             // this CTA's MMAs done with the K stage
-  uint64_t* pfull = bars + 2 * stages;         // P and alpha of every softmax warp of the cluster written
-  uint64_t* pempty = bars + 3 * stages;        // every CTA's MMAs done with the P stage
+  uint64_t* pfull = bars + 2 * stages;         // P and alpha of every head of the cluster in place
+  uint64_t* pempty = bars + 3 * stages;        // every CTA's MMAs done with the P stage, alphas read
   uint64_t* corr = bars + 4 * stages;          // accumulator corrected for this tile's new maxima
-  uint64_t* accfull = bars + 5 * stages;       // last MMA of an item completed
-  uint64_t* accempty = bars + 5 * stages + 1;  // epilogue finished reading the accumulator
+  uint64_t* pready = bars + 5 * stages;        // CL > 1: this CTA's P and alpha block written
+  uint64_t* accfull = bars + 6 * stages;       // last MMA of an item completed
+  uint64_t* accempty = bars + 6 * stages + 1;  // epilogue finished reading the accumulator
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.slot_off);
   int* s_nb = reinterpret_cast<int*>(smem + L.plan_off);
   int* s_rows = s_nb + (p.B + 1);
@@ -155,9 +166,13 @@ __global__ void __launch_bounds__(kTCThreads, 1)
       for (int s = 0; s < stages; ++s) {
         mbar_init(&full[s], 1);
         mbar_init(&empty[s], 1);
-        mbar_init(&pfull[s], kSoftmaxWarps * CL);
+        // CL = 1: the softmax warps arrive on pfull. CL > 1: they arrive on pready; the MMA
+        // thread then copies the block to the peers and arrives on pfull expecting the
+        // peers' blocks as transaction bytes.
+        mbar_init(&pfull[s], CL > 1 ? 1 : kSoftmaxWarps);
         mbar_init(&pempty[s], CL);
         mbar_init(&corr[s], 4);
+        mbar_init(&pready[s], kSoftmaxWarps);
       }
       mbar_init(accfull, 1);
       mbar_init(accempty, 4);
@@ -172,7 +187,6 @@ __global__ void __launch_bounds__(kTCThreads, 1)
     uint32_t* pz = reinterpret_cast<uint32_t*>(pst);
     for (uint32_t i = t; i < stages * pstage_bytes / 4u; i += kSoftmaxWarps * 32) pz[i] = 0u;
     for (int i = t; i < stages * kPRows; i += kSoftmaxWarps * 32) alpha_s[i] = 1.0f;
-    for (int i = t; i < stages; i += kSoftmaxWarps * 32) resc[i] = -1;
     fence_proxy_async_smem();
   }
   pdl_wait_primary();
@@ -221,7 +235,9 @@ __global__ void __launch_bounds__(kTCThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t kbase = smem_u32(kst), pbase = smem_u32(pst);
+      const uint32_t kbase = smem_u32(kst), pbase = smem_u32(pst), abase = smem_u32(alpha_s);
+      // this CTA's block of a P stage and of its alphas (rows [rank·64/CL, (rank+1)·64/CL))
+      constexpr uint32_t pblk = kPRows / CL * TT * 2, ablk = kPRows / CL * 4;
       int g = 0, ii = 0;
       bool ok = true;
       for (int item = group; item < n_items && ok; item += p.n_groups, ++ii) {
@@ -232,17 +248,49 @@ __global__ void __launch_bounds__(kTCThreads, 1)
         for (int t = 0; t < nt; ++t, ++g) {
           const int s = g % stages;
           const uint32_t ph = static_cast<uint32_t>(g / stages) & 1u;
-          // P of every head written (this CTA and its peers) and the K stage landed; the
-          // correction warps' pass is awaited only for a tile in which some head rescales
-          if (!mbar_wait<(CL > 1)>(&pfull[s], ph, p.status) || !mbar_wait(&full[s], ph, p.status) ||
-              (resc[s] == g && !mbar_wait(&corr[s], ph, p.status))) {
+          const uint32_t ka = kbase + s * kstage_bytes, pa = pbase + s * pstage_bytes;
+          if constexpr (CL > 1) {
+            // This CTA's rows of P and alpha are written: copy them into every peer (the
+            // copy completes on the peer's pfull) and expect the peers' rows on our pfull.
+            // The peers' previous use of the stage ended before the softmax warps wrote it.
+            if (!mbar_wait(&pready[s], ph, p.status)) {
+              ok = false;
+              break;
+            }
+            const uint32_t psrc = pa + rank * pblk, asrc = abase + (s * kPRows) * 4u + rank * ablk;
+            const uint32_t bar = smem_u32(&pfull[s]);
+#pragma unroll
+            for (int r = 1; r < CL; ++r) {
+              const uint32_t peer = (rank + r) % CL;
+              bulk_copy_to_peer(mapa_shared(psrc, peer), psrc, pblk, mapa_shared(bar, peer));
+              bulk_copy_to_peer(mapa_shared(asrc, peer), asrc, ablk, mapa_shared(bar, peer));
+            }
+            mbar_arrive_expect_tx(&pfull[s], (CL - 1) * (pblk + ablk));
+          }
+          // P of every head in place and the K stage landed
+          if (!mbar_wait<(CL > 1)>(&pfull[s], ph, p.status) || !mbar_wait(&full[s], ph, p.status)) {
+            ok = false;
+            break;
+          }
+          // the correction warps' pass comes first only in a tile in which some row rescales
+          // (all rows are checked: a straight run of loads measured faster than a loop over
+          // the rows in use)
+          bool resc = false;
+          if (t > 0) {
+            const float4* a4 = reinterpret_cast<const float4*>(alpha_s + s * kPRows);
+#pragma unroll
+            for (int i = 0; i < kPRows / 4; ++i) {
+              const float4 v = a4[i];
+              resc |= (v.x != 1.f) | (v.y != 1.f) | (v.z != 1.f) | (v.w != 1.f);
+            }
+          }
+          if (resc && !mbar_wait(&corr[s], ph, p.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const int r_lo = it.row0 + t * TT;
           const int nks = (min(TT, it.row1 - r_lo) + 15) / 16;
-          const uint32_t ka = kbase + s * kstage_bytes, pa = pbase + s * pstage_bytes;
           for (int kk = 0; kk < nks; ++kk) {
             const uint64_t ad = smem_desc(pa + kk * 256, 128, (TT / 8) * 128, kLayoutNone);
             for (int c = 0; c < dS; c += 256) {
@@ -254,6 +302,12 @@ __global__ void __launch_bounds__(kTCThreads, 1)
             }
           }
           umma_commit(&empty[s]);
+          // pempty releases the P stage and its alphas to every writer: the correction warps
+          // must have read the alphas first
+          if (!resc && !mbar_wait(&corr[s], ph, p.status)) {
+            ok = false;
+            break;
+          }
           if (CL > 1) umma_commit_mc(&pempty[s], static_cast<uint16_t>((1u << CL) - 1u));
           else umma_commit(&pempty[s]);
         }
@@ -268,9 +322,11 @@ __global__ void __launch_bounds__(kTCThreads, 1)
     }
   } else if (warp < 6) {
     // ------------------------------------------------------------ correction + epilogue warpgroup
-    // Lane l of quarter q holds head n = 4*(l % 16) + q in accumulator half l / 16.
+    // Lane l of quarter q holds P row 16 q + l % 16 (head n, or padding: n < 0) in accumulator
+    // half l / 16.
     const int quarter = warp & 3;
-    const int n = 4 * (lane & 15) + quarter, hf = lane >> 4;
+    const int prow = 16 * quarter + (lane & 15), hf = lane >> 4;
+    const int n = row_head(prow, CL, H_own);
     const int hcols = min(512, dS);  // columns per accumulator half
     const int my_cols = min(512, max(dS - 512 * hf, 0));
     const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
@@ -286,7 +342,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
           ok = false;
           break;
         }
-        const float alpha = (n < p.H) ? alpha_s[s * kPRows + n] : 1.f;
+        const float alpha = alpha_s[s * kPRows + prow];  // 1 in padding rows
         if (t > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
           // rescale this quarter's rows once the previous tile's MMAs have finished
           const int sp = (g - 1) % stages;
@@ -314,14 +370,14 @@ __global__ void __launch_bounds__(kTCThreads, 1)
       // epilogue: accumulator rows -> partial U[item][head][own columns]
       if (!__all_sync(0xffffffffu, mbar_wait(accfull, static_cast<uint32_t>(ii) & 1u, p.status))) break;
       tc_fence_after();
-      float* dst = p.ws_U + (static_cast<size_t>(item) * p.H + n) * p.d + col0 + 512 * hf;
+      float* dst = p.ws_U + (static_cast<size_t>(item) * p.H + max(n, 0)) * p.d + col0 + 512 * hf;
       // four 16-column loads in flight per wait (hcols and my_cols are multiples of 64)
       for (int c = 0; c < hcols; c += 64) {
         float v[4][16];
 #pragma unroll
         for (int j = 0; j < 4; ++j) tmem_ld16(tbase + c + 16 * j, v[j]);
         tmem_wait_ld();
-        if (n < p.H && c < my_cols) {
+        if (n >= 0 && c < my_cols) {
 #pragma unroll
           for (int j = 0; j < 4; ++j)
 #pragma unroll
@@ -345,7 +401,6 @@ __global__ void __launch_bounds__(kTCThreads, 1)
     const int row = TT == 32 ? (lane >> 3) + 4 * (lane & 7) : lane % TT, hslot = lane / TT;
     const uint32_t kbase = smem_u32(kst);
     const uint32_t pst_base = smem_u32(pst);
-    const uint32_t alpha_base = smem_u32(alpha_s);
     int g = 0;
     bool ok = true;
     for (int item = group; item < n_items && ok; item += p.n_groups) {
@@ -428,10 +483,9 @@ __global__ void __launch_bounds__(kTCThreads, 1)
           __syncwarp();
         }
 
-        // P stage s is free once the MMAs that read it (tile g - stages) finished in every CTA
-        // and this CTA's correction warps have read its alphas.
-        if (g >= stages && !__all_sync(0xffffffffu, mbar_wait<(CL > 1)>(&pempty[s], ph ^ 1u, p.status) &&
-                                                        mbar_wait(&corr[s], ph ^ 1u, p.status))) {
+        // P stage s is free once every CTA's MMAs and copies of tile g - stages finished with
+        // it and its correction warps read the alphas (each MMA thread commits after both).
+        if (g >= stages && !__all_sync(0xffffffffu, mbar_wait<(CL > 1)>(&pempty[s], ph ^ 1u, p.status))) {
           ok = false;
           break;
         }
@@ -530,8 +584,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
         for (int o = TT / 2; o > 0; o >>= 1)
 #pragma unroll
           for (int ps = 0; ps < NPASS; ++ps) mx[ps] = fmaxf(mx[ps], __shfl_xor_sync(0xffffffffu, mx[ps], o));
-        // Phase 3: lazy running max, P to shared memory (and the cluster peers)
-        bool rescaled = false;
+        // Phase 3: lazy running max, P and alpha to this CTA's rows of the stage
 #pragma unroll
         for (int ps = 0; ps < NPASS; ++ps) {
           const int k = ps * HPP + hslot;
@@ -544,10 +597,8 @@ __global__ void __launch_bounds__(kTCThreads, 1)
             alpha = exp2f(mref[ps] - mx[ps]);
             mref[ps] = mx[ps];
             lsum[ps] *= alpha;
-            rescaled = true;
           }
-          const int n = head0 + hh;
-          const int m = p_row(n);
+          const int m = p_row(head0 + hh, CL, H_own);
           const float pv = row < nvalid ? exp2f(sc[ps] - mref[ps]) : 0.f;
           const __nv_bfloat16 pb = __float2bfloat16_rn(pv);
           lsum[ps] += __bfloat162float(pb);
@@ -555,30 +606,12 @@ __global__ void __launch_bounds__(kTCThreads, 1)
                                static_cast<uint32_t>(((m >> 3) * (TT / 8) + (row >> 3)) * 128 + (m & 7) * 16 + (row & 7) * 2);
           const uint16_t bits = __bfloat16_as_ushort(pb);
           asm volatile("st.shared.u16 [%0], %1;" ::"r"(pst_base + off), "h"(bits) : "memory");
-#pragma unroll
-          for (int r = 1; r < CL; ++r) st_cluster_u16(mapa_shared(pst_base + off, (rank + r) % CL), bits);
-          if (row == 0) {
-            alpha_s[s * kPRows + n] = alpha;
-#pragma unroll
-            for (int r = 1; r < CL; ++r)
-              st_cluster_f32(mapa_shared(alpha_base + static_cast<uint32_t>((s * kPRows + n) * 4), (rank + r) % CL),
-                             alpha);
-          }
+          if (row == 0) alpha_s[s * kPRows + m] = alpha;
         }
-        if (__any_sync(0xffffffffu, rescaled) && lane == 0) {
-          resc[s] = g;
-#pragma unroll
-          for (int r = 1; r < CL; ++r)
-            st_cluster_f32(mapa_shared(smem_u32(const_cast<int*>(resc + s)), (rank + r) % CL), __int_as_float(g));
-        }
+        // the MMA operand (and, with peers, the block copy) reads P through the async proxy
         fence_proxy_async_smem();
-        if (CL > 1) fence_proxy_async_cluster();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&pfull[s]);
-#pragma unroll
-          for (int r = 1; r < CL; ++r) mbar_arrive_cluster(mapa_shared(smem_u32(&pfull[s]), (rank + r) % CL));
-        }
+        if (lane == 0) mbar_arrive(CL > 1 ? &pready[s] : &pfull[s]);
       }
       if (!ok) break;
       const size_t slot = static_cast<size_t>(item);

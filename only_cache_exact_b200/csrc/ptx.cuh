@@ -33,8 +33,15 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 // Arrive on an mbarrier given by a shared::cluster address (own or peer CTA).
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+// Bulk copy (async proxy) of `bytes` from this CTA's shared memory to a peer's;
+// the transfer completes as transaction bytes on the peer's mbarrier. Addresses
+// 16-byte aligned, size a multiple of 16. dst and mbar are cluster addresses.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src, uint32_t bytes,
+                                                  uint32_t mbar_cluster) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   dst_cluster),
+               "r"(src), "r"(bytes), "r"(mbar_cluster)
+               : "memory");
 }
 // Acquire at CTA scope: enough for TMA transactions, tcgen05 commits and
 // arrivals by this CTA's threads.
@@ -61,16 +68,27 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
   return ok != 0;
 }
 
-// Bounded wait for phase `parity` of `bar`. Gives up after about a second,
-// ORs SLIM_DEV_TIMEOUT into *status and returns false; the caller then
-// leaves its loop and the kernel tears down.
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Bounded wait for phase `parity` of `bar`. try_wait suspends the thread in
+// hardware until the phase completes (or a short hardware limit passes), so
+// the loop polls without sleeping: a sleep would delay every hand-off in the
+// pipeline by its wake-up time. After kWaitLimitNs of the global timer it ORs
+// SLIM_DEV_TIMEOUT into *status and returns false; the caller then leaves its
+// loop and the kernel tears down.
 template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status) {
   const uint32_t a = smem_u32(bar);
+  if (kCluster ? mbar_try_wait_cluster(a, parity) : mbar_try_wait(a, parity)) return true;
+  const uint64_t t0 = global_ns();
 #pragma unroll 1
-  for (uint32_t i = 0; i < kWaitSpinLimit; ++i) {
+  for (uint32_t i = 1;; ++i) {
     if (kCluster ? mbar_try_wait_cluster(a, parity) : mbar_try_wait(a, parity)) return true;
-    if (i >= 256) __nanosleep(64);
+    if ((i & 63u) == 0u && global_ns() - t0 > kWaitLimitNs) break;
   }
   atomicOr(status, SLIM_DEV_TIMEOUT);
   return false;
@@ -79,9 +97,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_
 // ------------------------------------------------------------------ fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ void fence_proxy_async_cluster() {
-  asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
 }
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
@@ -136,9 +151,6 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t local, uint32_t rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
   return r;
-}
-__device__ __forceinline__ void st_cluster_u16(uint32_t addr, uint16_t v) {
-  asm volatile("st.shared::cluster.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
 }
 __device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");

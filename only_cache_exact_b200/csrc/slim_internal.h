@@ -10,8 +10,8 @@
 
 namespace slim {
 
-// Bounded spin: ~16M polls with a 64 ns back-off ≈ 1-2 s before a wait gives up.
-constexpr uint32_t kWaitSpinLimit = 1u << 24;
+// A wait on an mbarrier gives up after this long (global timer, ns).
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
 // Work-list metadata written by the split kernel for the merge kernel:
 //   meta[0]          total number of work items

@@ -62,6 +62,23 @@ def oracle_out(c: Case, seqs=None) -> np.ndarray:
     return np.stack(res)
 
 
+def oracle_out_stored(c: Case, seqs=None) -> np.ndarray:
+    """Option (b) of the generation step evaluated exactly (float64 softmax and products) on the
+    operands the device stores: K and W_KV = W_K^(-1)·W_V rounded once to the cache type.
+    What remains between this and the device result is the kernels' own rounding (P in the
+    cache type, float32 sums); what separates it from oracle_out is the method's storage
+    precision, which W_KV amplifies by the conditioning of W_K."""
+    seqs = range(c.B) if seqs is None else seqs
+    wkv = synth.round_to(O.wkv_solve(c.w.W_K, c.w.W_V), c.dtype)
+    res = []
+    for b in seqs:
+        K = synth.round_to(O.project(c.X[b], c.w.W_K), c.dtype)
+        if c.append:
+            K = np.vstack([K, synth.round_to(c.k_new64[b], c.dtype)[None]])
+        res.append(O.slim_decode_b(c.q64[b], K, wkv, c.H))
+    return np.stack(res)
+
+
 class GpuState:
     """Device buffers of a case: cache filled by slim_prefill_k, W_KV, inputs, workspace."""
 

@@ -1,6 +1,7 @@
 """GPU parity of slim_decode_step (both orderings) and slim_prefill_k against the float64 oracle.
 
-Tolerances: bf16 caches, relative L2 per (sequence, head) <= 2e-2; fp32
+Tolerances: bf16 caches, relative L2 per (sequence, head) <= 2e-2 against exact
+MHA, or <= 1e-2 against option (b) evaluated exactly on the stored operands; fp32
 cache (the fp32 workload), max-abs <= 2e-3. Integer/byte results (lengths,
 appended cache rows, status bits) are compared exactly.
 """
@@ -8,7 +9,7 @@ import numpy as np
 import pytest
 import torch
 
-from tests.gpu_cases import GpuState, make_case, oracle_out, rel_l2_per_head
+from tests.gpu_cases import GpuState, make_case, oracle_out, oracle_out_stored, rel_l2_per_head
 from oracle import slim_oracle as O
 from only_cache_exact_b200 import synth
 
@@ -16,6 +17,7 @@ pytestmark = pytest.mark.gpu
 
 TOL_BF16 = 2e-2
 TOL_F32 = 2e-3
+TOL_STORED = 1e-2  # bf16 P and float32 sums against float64 on the same stored operands
 
 
 @pytest.fixture(scope="module")
@@ -55,15 +57,22 @@ def test_cross_attention_fixed_cache_d1280(S):
     assert torch.equal(g.lens.cpu(), torch.from_numpy(c.lens))
 
 
-def test_d4096_two_cta_cluster(S):
+def test_d4096_four_cta_cluster(S):
     c = make_case(4096, 32, lens=[700, 333, 64], cap=800, seed=3)
     g = GpuState(c, S)
     _check_bf16(g.step(S.SLIM_VARIANT_B), oracle_out(c), c.H)
 
 
-def test_rising_scores_force_rescale(S):
-    """Later rows scaled up so each head's running max grows by far more than 2^8 across tiles."""
-    c = make_case(1024, 16, lens=[600, 257], cap=700, seed=4)
+@pytest.mark.parametrize("d,H", [(1024, 16), (1280, 20), (4096, 32)])
+def test_rising_scores_force_rescale(S, d, H):
+    """Later rows scaled up so each head's running max grows by far more than 2^8 across tiles
+    (one CTA per item at d=1024; clusters of 2 and 4 CTAs exchanging P and alpha above).
+
+    The softmax is sharply peaked here, so the bf16 cache's rounding, amplified through W_KV,
+    moves some heads by a few percent from exact MHA whatever the kernel does (3.6% and 6.6%
+    at d=1280 and d=4096 with float64 arithmetic on the stored operands). The kernels are
+    therefore held to the stored-operand evaluation of option (b) at a tighter bound."""
+    c = make_case(d, H, lens=[600, 257], cap=700, seed=4)
     for b in range(c.B):
         n = len(c.X[b])
         scale = np.linspace(0.2, 6.0, n)[:, None]
@@ -71,10 +80,10 @@ def test_rising_scores_force_rescale(S):
     c.x_new = synth.round_to(c.x_new * 3.0, "bf16")
     c.q64 = c.x_new @ c.w.W_Q
     c.k_new64 = c.x_new @ c.w.W_K
-    g = GpuState(c, S)
-    _check_bf16(g.step(S.SLIM_VARIANT_B), oracle_out(c), c.H)
-    g2 = GpuState(c, S)
-    _check_bf16(g2.step(S.SLIM_VARIANT_A), oracle_out(c), c.H)
+    ref = oracle_out_stored(c)
+    for v in (S.SLIM_VARIANT_B, S.SLIM_VARIANT_A):
+        err = rel_l2_per_head(GpuState(c, S).step(v), ref, c.H)
+        assert err.max() <= TOL_STORED, (v, err.max(), np.unravel_index(err.argmax(), err.shape))
 
 
 def test_empty_and_single_row(S):
