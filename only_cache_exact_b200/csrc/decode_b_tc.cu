@@ -12,7 +12,7 @@
 //
 // A cluster of CL CTAs shares one work item; CTA r owns the columns
 // [r·dS, (r+1)·dS), dS = d/CL <= 1024, and the heads whose columns lie there.
-// Per CTA (14 warps):
+// Per CTA (16 warps):
 //   warp 0       TMA producer: a K tile is TT rows x dS columns, one 3-D box
 //                per 16-row slab (128-byte swizzle), evict-first in L2.
 //   warp 1       MMA issuer: U[heads, own columns] += P[heads, rows] · K[rows,
@@ -20,21 +20,24 @@
 //                N <= 256 (columns), K = 16 rows; the K slab is read in place
 //                as the MN-major B operand. Two M=64 accumulators interleave in
 //                TMEM (lane offsets 0 and 16), so 1024 columns fit in the 512
-//                TMEM columns. With CL > 1 it first sends this CTA's rows of
-//                P and alpha to every peer as one bulk shared-to-shared copy
-//                each (completing on the peer's mbarrier): one hop through
-//                distributed shared memory per tile, no cluster-scope fence.
+//                TMEM columns.
 //   warps 2..5   correction and epilogue: the lazy online-softmax rescale of
 //                the accumulator rows whose max grew by more than 2^8 (the MMA
 //                warp waits for this pass first only on tiles with a rescaled
 //                row), and TMEM -> partials in global memory.
-//   warps 6..13  scores: per head, q_h·K_t on the CUDA cores (32-row tiles: a
+//   warps 6..15  scores: per head, q_h·K_t on the CUDA cores (32-row tiles: a
 //                lane multiplies one 16-byte chunk of 8 rows by q held in
 //                registers, a butterfly over the 8 chunk lanes sums the rows;
 //                16-row tiles: one row per lane, q broadcast from shared
 //                memory), fp32 accumulation, running max, P in bf16 and the
-//                rescale factors to this CTA's rows of the stage. The tensor
-//                pipe is left to the P·K MMAs.
+//                rescale factors to this CTA's rows of the stage. With CL > 1
+//                the same warps store those rows into every peer with st.async
+//                (16 bytes of P per store), which completes the bytes on the
+//                peer's mbarrier: no fence and no round trip on the sending
+//                side, and the stores do not queue behind the TMA unit's K
+//                loads as a bulk copy would. The tensor pipe is left to the
+//                P·K MMAs. Ten warps, so that 10 heads (d=1280, H=20 split
+//                over two CTAs) take one warp each.
 // Every mbarrier wait is bounded; a timeout sets SLIM_DEV_TIMEOUT and the
 // kernel drains its copies and MMAs, frees TMEM and returns.
 #include <cuda_bf16.h>
@@ -51,7 +54,7 @@ namespace slim {
 // A head's running max may grow by this much (log2 units) before its TMEM row
 // is rescaled: P stays <= 2^8 in bf16 and no precision is lost.
 constexpr float kLazyRescaleLog2 = 8.f;
-constexpr int kSoftmaxWarps = 8;
+constexpr int kSoftmaxWarps = 10;
 constexpr int kTCThreads = (6 + kSoftmaxWarps) * 32;
 constexpr int kMaxColsPerCTA = 1024;  // two interleaved M=64 accumulators x 512 TMEM columns
 constexpr int kPRows = 64;            // M of the P·K MMA: heads, padded
@@ -95,7 +98,7 @@ __host__ __device__ inline TCSmem tc_smem_layout(int CL, int TT, int d, int stag
   o += dS * 4u;
   o = (o + 7u) & ~7u;
   s.bar_off = o;
-  o += (6u * stages + 2u) * 8u;
+  o += (5u * stages + 2u) * 8u;
   s.slot_off = o;
   o += 16u;
   s.plan_off = o;
@@ -144,9 +147,8 @@ __global__ void __launch_bounds__(kTCThreads, 1)
   uint64_t* pfull = bars + 2 * stages;         // P and alpha of every head of the cluster in place
   uint64_t* pempty = bars + 3 * stages;        // every CTA's MMAs done with the P stage, alphas read
   uint64_t* corr = bars + 4 * stages;          // accumulator corrected for this tile's new maxima
-  uint64_t* pready = bars + 5 * stages;        // CL > 1: this CTA's P and alpha block written
-  uint64_t* accfull = bars + 6 * stages;       // last MMA of an item completed
-  uint64_t* accempty = bars + 6 * stages + 1;  // epilogue finished reading the accumulator
+  uint64_t* accfull = bars + 5 * stages;       // last MMA of an item completed
+  uint64_t* accempty = bars + 5 * stages + 1;  // epilogue finished reading the accumulator
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.slot_off);
   int* s_nb = reinterpret_cast<int*>(smem + L.plan_off);
   int* s_rows = s_nb + (p.B + 1);
@@ -166,13 +168,11 @@ __global__ void __launch_bounds__(kTCThreads, 1)
       for (int s = 0; s < stages; ++s) {
         mbar_init(&full[s], 1);
         mbar_init(&empty[s], 1);
-        // CL = 1: the softmax warps arrive on pfull. CL > 1: they arrive on pready; the MMA
-        // thread then copies the block to the peers and arrives on pfull expecting the
-        // peers' blocks as transaction bytes.
-        mbar_init(&pfull[s], CL > 1 ? 1 : kSoftmaxWarps);
+        // one arrival per softmax warp; with peers, one of them also expects the peers'
+        // P rows and alphas as transaction bytes
+        mbar_init(&pfull[s], kSoftmaxWarps);
         mbar_init(&pempty[s], CL);
         mbar_init(&corr[s], 4);
-        mbar_init(&pready[s], kSoftmaxWarps);
       }
       mbar_init(accfull, 1);
       mbar_init(accempty, 4);
@@ -235,9 +235,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t kbase = smem_u32(kst), pbase = smem_u32(pst), abase = smem_u32(alpha_s);
-      // this CTA's block of a P stage and of its alphas (rows [rank·64/CL, (rank+1)·64/CL))
-      constexpr uint32_t pblk = kPRows / CL * TT * 2, ablk = kPRows / CL * 4;
+      const uint32_t kbase = smem_u32(kst), pbase = smem_u32(pst);
       int g = 0, ii = 0;
       bool ok = true;
       for (int item = group; item < n_items && ok; item += p.n_groups, ++ii) {
@@ -249,29 +247,12 @@ __global__ void __launch_bounds__(kTCThreads, 1)
           const int s = g % stages;
           const uint32_t ph = static_cast<uint32_t>(g / stages) & 1u;
           const uint32_t ka = kbase + s * kstage_bytes, pa = pbase + s * pstage_bytes;
-          if constexpr (CL > 1) {
-            // This CTA's rows of P and alpha are written: copy them into every peer (the
-            // copy completes on the peer's pfull) and expect the peers' rows on our pfull.
-            // The peers' previous use of the stage ended before the softmax warps wrote it.
-            if (!mbar_wait(&pready[s], ph, p.status)) {
-              ok = false;
-              break;
-            }
-            const uint32_t psrc = pa + rank * pblk, asrc = abase + (s * kPRows) * 4u + rank * ablk;
-            const uint32_t bar = smem_u32(&pfull[s]);
-#pragma unroll
-            for (int r = 1; r < CL; ++r) {
-              const uint32_t peer = (rank + r) % CL;
-              bulk_copy_to_peer(mapa_shared(psrc, peer), psrc, pblk, mapa_shared(bar, peer));
-              bulk_copy_to_peer(mapa_shared(asrc, peer), asrc, ablk, mapa_shared(bar, peer));
-            }
-            mbar_arrive_expect_tx(&pfull[s], (CL - 1) * (pblk + ablk));
-          }
           // P of every head in place and the K stage landed
           if (!mbar_wait<(CL > 1)>(&pfull[s], ph, p.status) || !mbar_wait(&full[s], ph, p.status)) {
             ok = false;
             break;
           }
+          if constexpr (CL > 1) fence_proxy_async_acquire_peers();  // peers' rows, for the MMA
           // the correction warps' pass comes first only in a tile in which some row rescales
           // (all rows are checked: a straight run of loads measured faster than a loop over
           // the rows in use)
@@ -608,10 +589,51 @@ __global__ void __launch_bounds__(kTCThreads, 1)
           asm volatile("st.shared.u16 [%0], %1;" ::"r"(pst_base + off), "h"(bits) : "memory");
           if (row == 0) alpha_s[s * kPRows + m] = alpha;
         }
-        // the MMA operand (and, with peers, the block copy) reads P through the async proxy
+        // the MMA operand reads P through the async proxy
         fence_proxy_async_smem();
+        if constexpr (CL > 1) {
+          // every peer gets this warp's rows of P (16-byte chunks of 8 rows) and alphas by
+          // stores that complete on the peer's pfull
+          __syncwarp();
+          constexpr int kChunks = HPW * (TT / 8);
+          if (lane < kChunks || lane >= 32 - HPW) {
+            const int k = lane < kChunks ? lane / (TT / 8) : 31 - lane;
+            const int hh = sw + kSoftmaxWarps * k;
+            if (hh < H_own) {
+              const int m = p_row(head0 + hh, CL, H_own);
+              const uint32_t bar = smem_u32(&pfull[s]);
+              if (lane < kChunks) {
+                const uint32_t off = static_cast<uint32_t>(s) * pstage_bytes +
+                                     static_cast<uint32_t>(((m >> 3) * (TT / 8) + lane % (TT / 8)) * 128 + (m & 7) * 16);
+                uint4 v;
+                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                             : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                             : "r"(pst_base + off));
+#pragma unroll
+                for (int r = 1; r < CL; ++r) {
+                  const uint32_t peer = (rank + r) % CL;
+                  st_async_v4(mapa_shared(pst_base + off, peer), v, mapa_shared(bar, peer));
+                }
+              } else {
+                const uint32_t a = smem_u32(alpha_s + s * kPRows + m);
+                const uint32_t v = __float_as_uint(alpha_s[s * kPRows + m]);
+#pragma unroll
+                for (int r = 1; r < CL; ++r) {
+                  const uint32_t peer = (rank + r) % CL;
+                  st_async_b32(mapa_shared(a, peer), v, mapa_shared(bar, peer));
+                }
+              }
+            }
+          }
+        }
         __syncwarp();
-        if (lane == 0) mbar_arrive(CL > 1 ? &pready[s] : &pfull[s]);
+        if (lane == 0) {
+          // the peers' rows arrive as transaction bytes: H_own heads x (TT P values + alpha) each
+          if (CL > 1 && sw == 0)
+            mbar_arrive_expect_tx(&pfull[s], static_cast<uint32_t>((CL - 1) * H_own * (TT * 2 + 4)));
+          else
+            mbar_arrive(&pfull[s]);
+        }
       }
       if (!ok) break;
       const size_t slot = static_cast<size_t>(item);

@@ -33,15 +33,22 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 // Arrive on an mbarrier given by a shared::cluster address (own or peer CTA).
-// Bulk copy (async proxy) of `bytes` from this CTA's shared memory to a peer's;
-// the transfer completes as transaction bytes on the peer's mbarrier. Addresses
-// 16-byte aligned, size a multiple of 16. dst and mbar are cluster addresses.
-__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cluster, uint32_t src, uint32_t bytes,
-                                                  uint32_t mbar_cluster) {
-  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   dst_cluster),
-               "r"(src), "r"(bytes), "r"(mbar_cluster)
+// Store into a peer CTA's shared memory (cluster addresses) that completes its
+// bytes on the peer's mbarrier; no fence or arrival needed on this side.
+__device__ __forceinline__ void st_async_v4(uint32_t addr, uint4 v, uint32_t mbar) {
+  asm volatile("st.async.weak.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(addr),
+               "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(mbar)
                : "memory");
+}
+__device__ __forceinline__ void st_async_b32(uint32_t addr, uint32_t v, uint32_t mbar) {
+  asm volatile("st.async.weak.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(addr), "r"(v),
+               "r"(mbar)
+               : "memory");
+}
+// After an mbarrier wait has observed peers' st.async data: makes it visible to
+// this thread's later async-proxy reads (tcgen05.mma operands).
+__device__ __forceinline__ void fence_proxy_async_acquire_peers() {
+  asm volatile("fence.proxy.async::generic.acquire.sync_restrict::shared::cluster.cluster;" ::: "memory");
 }
 // Acquire at CTA scope: enough for TMA transactions, tcgen05 commits and
 // arrivals by this CTA's threads.
