@@ -43,6 +43,7 @@
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <cstdlib>
 #include <map>
 #include <mutex>
 #include <utility>
@@ -695,12 +696,26 @@ uint32_t pow2_cols(uint32_t c) {
   return r;
 }
 
+// SLIM_SPLIT_CLUSTER=1|2|4 in the environment forces the cluster size of the
+// split kernel where that size is valid for the shape (a tuning knob; read once).
+int forced_cluster() {
+  static const int v = [] {
+    const char* e = std::getenv("SLIM_SPLIT_CLUSTER");
+    const int c = e ? std::atoi(e) : 0;
+    return (c == 1 || c == 2 || c == 4) ? c : 0;
+  }();
+  return v;
+}
+
 bool pick_config(int B, int d, int H, TCConfig* out) {
   if (H <= 0 || d % H || H > kPRows) return false;
   const int dh = d / H;
   if (dh != 64 && dh != 128) return false;
   const int smem_cap = max_smem_optin();
+  const int force = forced_cluster();
+  for (int pass = force ? 0 : 1; pass < 2; ++pass)
   for (int CL = 1; CL <= 4; CL *= 2) {
+    if (pass == 0 && CL != force) continue;
     if (d % (64 * CL) || H % CL || (d / CL) % dh || d / CL > kMaxColsPerCTA) continue;
     const int H_own = H / CL;
     const int HPW = (H_own + kSoftmaxWarps - 1) / kSoftmaxWarps;

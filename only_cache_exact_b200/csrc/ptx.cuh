@@ -147,6 +147,15 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* map, int32_t 
       : "memory");
 }
 
+// Untiled bulk copy global -> this CTA's shared memory (no multicast); both addresses 16-byte
+// aligned, bytes a multiple of 16; completes `bytes` on `bar`.
+__device__ __forceinline__ void bulk_load_g2s(void* sdst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(sdst)),
+               "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
 // ------------------------------------------------------------------ cluster
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;

@@ -318,6 +318,184 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
   }
 }
 
+// ---------------------------------------------------------------------------- one-sequence merge
+// The same merge and projection for shapes whose head slice of W_KV fits in shared memory
+// (d_h = 64, d <= 1280) and whose B x H CTAs fit in one wave: CTA (h, b) owns head h of
+// sequence b entirely, so no cluster reduction follows the projection.
+//   * Before the split kernel's results are awaited: W_KV[:, h-cols] (d rows x 128 bytes,
+//     128-byte swizzled) by TMA.
+//   * The item range of sequence b, then in one round trip the items' m and l and their U rows
+//     of head h (one bulk copy of d floats per item, completing on an mbarrier).
+//   * Every thread holds the columns tid + 256 i of ū = Σ_c 2^(m_c - M) U_c / Σ_c 2^(m_c - M) l_c
+//     and multiplies them by the matching W_KV rows (conflict-free swizzled 16-byte reads);
+//     a butterfly over the warp leaves two of the 64 outputs per lane, and 64 threads add the
+//     eight warps' sums.
+struct MergeLeanParams {
+  const float* U;
+  const float* m;
+  const float* l;
+  const int32_t* meta;
+  float* out;
+  int32_t* lens;
+  int32_t* status;
+  int B, d, H, max_items;
+  int cap_items;  // U rows staged per round
+};
+
+constexpr int kLeanThreads = 256;
+constexpr int kLeanDh = 64;
+constexpr int kLeanMaxCols = 1280;
+constexpr int kLeanCols = kLeanMaxCols / kLeanThreads;  // columns of ū per thread
+
+struct LeanSmem {
+  uint32_t w, u, ml, red, bars, total;
+};
+__host__ __device__ inline LeanSmem lean_smem_layout(int d, int cap_items, int max_items) {
+  LeanSmem s;
+  uint32_t o = 0;
+  s.w = o;  // [d rows][64 bf16], 128-byte swizzle (1024-byte aligned base)
+  o += up_to(static_cast<uint32_t>(d) * kLeanDh * 2u, 1024u);
+  s.u = o;  // [cap_items][d] fp32
+  o += static_cast<uint32_t>(cap_items) * d * 4u;
+  s.ml = o;  // m then l of the sequence's items
+  o += up_to(2u * static_cast<uint32_t>(max_items) * 4u, 16u);
+  s.red = o;  // [8 warps][64]
+  o += (kLeanThreads / 32) * kLeanDh * 4u;
+  s.bars = o;
+  o += 32u;
+  s.total = o + 1024u;  // slack to align the base to 1024 bytes
+  return s;
+}
+
+__global__ void __launch_bounds__(kLeanThreads, 1)
+    merge_lean_kernel(const __grid_constant__ CUtensorMap wmap, const MergeLeanParams p) {
+  extern __shared__ uint8_t lsm_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(lsm_raw) + 1023) & ~uintptr_t(1023));
+  const LeanSmem L = lean_smem_layout(p.d, p.cap_items, p.max_items);
+  const int h = blockIdx.x, b = blockIdx.y, d = p.d;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  float* us = reinterpret_cast<float*>(sm + L.u);
+  float* ms = reinterpret_cast<float*>(sm + L.ml);
+  float* ls = ms + p.max_items;
+  float* red = reinterpret_cast<float*>(sm + L.red);
+  uint64_t* wbar = reinterpret_cast<uint64_t*>(sm + L.bars);
+  uint64_t* ubar = wbar + 1;
+  int* rng = reinterpret_cast<int*>(wbar + 2);
+
+  if (tid == 0) {
+    mbar_init(wbar, 1);
+    mbar_init(ubar, 1);
+    fence_barrier_init();
+    tma_prefetch_desc(&wmap);
+    mbar_arrive_expect_tx(wbar, static_cast<uint32_t>(d) * kLeanDh * 2u);
+    for (int y = 0; y < d; y += 256)
+      tma_load_2d(sm + L.w + static_cast<size_t>(y) * 128, &wmap, h * kLeanDh, y, wbar, l2_policy_evict_last());
+  }
+  __syncthreads();
+  pdl_wait_primary();
+  pdl_launch_dependents();
+
+  if (tid < 2) rng[tid] = __ldcg(p.meta + 1 + b + tid);
+  if (h == 0 && tid == 32 && (__ldcg(p.meta + 2 + p.B + b) & kSeqAppend)) p.lens[b] += 1;
+  __syncthreads();
+  const int lo = rng[0], n = rng[1] - lo;
+  const uint32_t row_bytes = static_cast<uint32_t>(d) * 4u;
+  auto stage = [&](int r0) {  // one thread: U rows of items lo + r0 .. into shared memory
+    const int nr = min(n - r0, p.cap_items);
+    mbar_arrive_expect_tx(ubar, static_cast<uint32_t>(nr) * row_bytes);
+    for (int c = 0; c < nr; ++c)
+      bulk_load_g2s(us + static_cast<size_t>(c) * d, p.U + (static_cast<size_t>(lo + r0 + c) * p.H + h) * d,
+                    row_bytes, ubar);
+  };
+  if (tid == 0 && n > 0) stage(0);
+  for (int c = tid; c < n; c += kLeanThreads) {
+    ms[c] = __ldcg(p.m + static_cast<size_t>(lo + c) * p.H + h);
+    ls[c] = __ldcg(p.l + static_cast<size_t>(lo + c) * p.H + h);
+  }
+  __syncthreads();
+
+  // merge weights, computed by every thread from the shared m, l
+  float M = -INFINITY;
+  for (int c = 0; c < n; ++c) M = fmaxf(M, ms[c]);
+  float S = 0.f;
+  for (int c = 0; c < n; ++c) S = fmaf(exp2f(ms[c] - M), ls[c], S);
+  const float inv = S > 0.f ? 1.f / S : 0.f;
+
+  float ub[kLeanCols];
+#pragma unroll
+  for (int i = 0; i < kLeanCols; ++i) ub[i] = 0.f;
+  bool ok = true;
+  uint32_t ph = 0;
+  for (int r0 = 0; r0 < n; r0 += p.cap_items, ph ^= 1u) {
+    ok = __syncthreads_and(mbar_wait(ubar, ph, p.status));
+    if (!ok) break;
+    const int nr = min(n - r0, p.cap_items);
+    for (int c = 0; c < nr; ++c) {
+      const float w = exp2f(ms[r0 + c] - M) * inv;
+      const float* row = us + static_cast<size_t>(c) * d;
+#pragma unroll
+      for (int i = 0; i < kLeanCols; ++i) {
+        const int col = tid + kLeanThreads * i;
+        if (col < d) ub[i] = fmaf(w, row[col], ub[i]);
+      }
+    }
+    if (r0 + p.cap_items < n) {
+      __syncthreads();  // every thread is done with the staged rows
+      if (tid == 0) stage(r0 + p.cap_items);
+    }
+  }
+  ok = __syncthreads_and(ok && mbar_wait(wbar, 0u, p.status));
+
+  // o[j] = Σ_rows ū[row] W[row][j]: this thread's rows, all 64 outputs
+  float acc[kLeanDh];
+#pragma unroll
+  for (int j = 0; j < kLeanDh; ++j) acc[j] = 0.f;
+  const uint32_t wbase = smem_u32(sm + L.w);
+#pragma unroll
+  for (int i = 0; i < kLeanCols; ++i) {
+    const int row = tid + kLeanThreads * i;
+    if (row < d) {
+      const float u = ub[i];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        uint4 v;
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                     : "r"(wbase + static_cast<uint32_t>(row) * 128u + ((static_cast<uint32_t>(k ^ (row & 7))) << 4)));
+        acc[8 * k + 0] = fmaf(u, bf16lo(v.x), acc[8 * k + 0]);
+        acc[8 * k + 1] = fmaf(u, bf16hi(v.x), acc[8 * k + 1]);
+        acc[8 * k + 2] = fmaf(u, bf16lo(v.y), acc[8 * k + 2]);
+        acc[8 * k + 3] = fmaf(u, bf16hi(v.y), acc[8 * k + 3]);
+        acc[8 * k + 4] = fmaf(u, bf16lo(v.z), acc[8 * k + 4]);
+        acc[8 * k + 5] = fmaf(u, bf16hi(v.z), acc[8 * k + 5]);
+        acc[8 * k + 6] = fmaf(u, bf16lo(v.w), acc[8 * k + 6]);
+        acc[8 * k + 7] = fmaf(u, bf16hi(v.w), acc[8 * k + 7]);
+      }
+    }
+  }
+  // butterfly reduce-scatter over the warp: after the stage with offset o a lane keeps the half
+  // of its values selected by lane bit o, summed with its partner's copy; lane l ends with the
+  // warp sums of outputs 2l and 2l + 1
+#pragma unroll
+  for (int s = kLeanDh / 2, o = 16; s >= 2; s >>= 1, o >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < s; ++i) {
+      const float send = up ? acc[i] : acc[i + s];
+      const float keep = up ? acc[i + s] : acc[i];
+      acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  *reinterpret_cast<float2*>(red + warp * kLeanDh + 2 * lane) = make_float2(acc[0], acc[1]);
+  __syncthreads();
+  if (tid < kLeanDh) {
+    float a = 0.f;
+#pragma unroll
+    for (int w = 0; w < kLeanThreads / 32; ++w) a += red[w * kLeanDh + tid];
+    p.out[static_cast<size_t>(b) * d + h * kLeanDh + tid] = (ok && n > 0) ? a : 0.f;
+  }
+}
+
 // ---------------------------------------------------------------------------- ordering (a) merge
 struct ReduceAParams {
   const float* O;
@@ -398,8 +576,65 @@ bool pick_merge(int B, int d, int H, int esz, int max_items, MergeConfig* c) {
 
 }  // namespace
 
+namespace {
+
+// Rows of U staged per round by merge_lean_kernel for this shape, 0 if it does not apply.
+int lean_cap_items(int B, int d, int H, int dtype, int max_items) {
+  if (dtype != SLIM_BF16 || H * kLeanDh != d || d % kLeanThreads || d > kLeanMaxCols) return 0;
+  if (static_cast<long long>(B) * H > num_sms()) return 0;  // one wave (one CTA per SM)
+  const int optin = max_smem_optin();
+  const uint32_t fixed = lean_smem_layout(d, 0, max_items).total;
+  if (fixed >= static_cast<uint32_t>(optin)) return 0;
+  const int cap = std::min(32, static_cast<int>((static_cast<uint32_t>(optin) - fixed) / (static_cast<uint32_t>(d) * 4u)));
+  return cap >= 4 ? cap : 0;
+}
+
+cudaError_t launch_merge_lean(const DecodeArgs& a, const SplitWorkspace& ws, int cap, bool pdl, cudaStream_t st,
+                              int* launches) {
+  CUtensorMap wmap;
+  const uint64_t dims[2] = {static_cast<uint64_t>(a.d), static_cast<uint64_t>(a.d)};
+  const uint64_t strides[1] = {static_cast<uint64_t>(a.d) * 2u};
+  const uint32_t box[2] = {static_cast<uint32_t>(kLeanDh), 256u};
+  if (!encode_tmap(&wmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.w_kv, dims, strides, box, true))
+    return cudaErrorInvalidValue;
+  MergeLeanParams p;
+  p.U = ws.U;
+  p.m = ws.m;
+  p.l = ws.l;
+  p.meta = ws.meta;
+  p.out = a.out;
+  p.lens = a.lens;
+  p.status = a.status;
+  p.B = a.B;
+  p.d = a.d;
+  p.H = a.H;
+  p.max_items = ws.max_items;
+  p.cap_items = cap;
+  const uint32_t smem = lean_smem_layout(a.d, cap, ws.max_items).total;
+  cudaError_t e = cudaFuncSetAttribute(merge_lean_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(a.H), static_cast<unsigned>(a.B), 1);
+  cfg.blockDim = dim3(kLeanThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, merge_lean_kernel, wmap, p);
+  if (e == cudaSuccess && launches) ++*launches;
+  return e;
+}
+
+}  // namespace
+
 cudaError_t launch_reduce_b(const DecodeArgs& a, const SplitWorkspace& ws, bool pdl, cudaStream_t st,
                             int* launches) {
+  if (const int cap = lean_cap_items(a.B, a.d, a.H, a.dtype, ws.max_items))
+    return launch_merge_lean(a, ws, cap, pdl, st, launches);
   const int esz = a.dtype == SLIM_BF16 ? 2 : 4;
   const int d_h = a.d / a.H;
   MergeConfig c;
