@@ -124,6 +124,38 @@ __host__ __device__ inline int row_head(int i, int CL, int H_own) {
   return j < H_own ? r * H_own + j : -1;
 }
 
+// Softmax warps are warps 6 .. 6 + kSoftmaxWarps - 1; warp w issues on sub-partition w % 4.
+// The SMSP-balanced assignment gives head j to sub-partition j % 4 and, within it, to its
+// softmax warps in turn, so every sub-partition issues about H_own / 4 heads' score work (the
+// plain assignment, heads sw, sw + kSoftmaxWarps, ..., leaves 5 of 16 heads on two of them).
+// It is used when no warp then needs more than HPW heads.
+__host__ __device__ inline void smsp_warps(int x, int* first, int* len) {
+  *first = 6 + ((x + 2) & 3);
+  *len = (6 + kSoftmaxWarps - *first + 3) / 4;
+}
+__host__ __device__ inline bool balanced_heads_fit(int H_own, int HPW) {
+  for (int x = 0; x < 4; ++x) {
+    int first, len;
+    smsp_warps(x, &first, &len);
+    const int n = H_own > x ? (H_own - x + 3) / 4 : 0;
+    if ((n + len - 1) / len > HPW) return false;
+  }
+  return true;
+}
+// Head of softmax warp sw in slot k, or H_own when the slot is empty.
+__host__ __device__ inline int softmax_head(int sw, int k, int H_own, bool balanced) {
+  int j;
+  if (balanced) {
+    const int w = sw + 6, x = w & 3;
+    int first, len;
+    smsp_warps(x, &first, &len);
+    j = x + 4 * ((w - first) / 4 + len * k);
+  } else {
+    j = sw + kSoftmaxWarps * k;
+  }
+  return j < H_own ? j : H_own;
+}
+
 template <int CL, int TT, int DHB, int HPW>
 __global__ void __launch_bounds__(kTCThreads, 1)
     decode_b_tc_kernel(const __grid_constant__ CUtensorMap kmap, const DecodeTCParams p) {
@@ -374,7 +406,8 @@ __global__ void __launch_bounds__(kTCThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ score / softmax warps
-    const int sw = warp - 6;  // heads sw, sw + 8, ... of this CTA
+    const int sw = warp - 6;
+    const bool hbal = balanced_heads_fit(H_own, HPW);
     constexpr int HPP = 32 / TT;                  // heads per pass (one row per lane)
     constexpr int NPASS = (HPW + HPP - 1) / HPP;  // passes over this warp's heads
     // TT = 32: lane (chunk c = lane % 8, row group rg = lane / 8) multiplies 16-byte chunk c of
@@ -383,6 +416,13 @@ __global__ void __launch_bounds__(kTCThreads, 1)
     const int row = TT == 32 ? (lane >> 3) + 4 * (lane & 7) : lane % TT, hslot = lane / TT;
     const uint32_t kbase = smem_u32(kst);
     const uint32_t pst_base = smem_u32(pst);
+    int mrow[NPASS];  // P row of this lane's head in each pass
+#pragma unroll
+    for (int ps = 0; ps < NPASS; ++ps) {
+      const int k = ps * HPP + hslot;
+      const int hh = softmax_head(sw, k, H_own, hbal);
+      mrow[ps] = (k < HPW && hh < H_own) ? p_row(head0 + hh, CL, H_own) : 0;
+    }
     int g = 0;
     bool ok = true;
     for (int item = group; item < n_items && ok; item += p.n_groups) {
@@ -393,7 +433,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
       // q of this warp's heads to shared memory (read back as broadcasts, or kept in registers
       // for this lane's chunks when TT = 32)
       float mref[NPASS], lsum[NPASS];  // running max and sum of this lane's head in each pass
-      float qr[TT == 32 ? HPW : 1][DHB][8];
+      uint64_t qp[TT == 32 ? HPW : 1][DHB][4];  // q pairs of this lane's chunk (fma.rn.f32x2 operands)
 #pragma unroll
       for (int ps = 0; ps < NPASS; ++ps) {
         mref[ps] = -INFINITY;
@@ -402,7 +442,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
       __syncwarp();
 #pragma unroll
       for (int k = 0; k < HPW; ++k) {
-        const int hh = sw + kSoftmaxWarps * k;
+        const int hh = softmax_head(sw, k, H_own, hbal);
         if (hh < H_own) {
           const float* src = p.q + static_cast<size_t>(b) * p.d + col0 + hh * DH;
           for (int i = lane; i < DH / 4; i += 32)
@@ -413,13 +453,15 @@ __global__ void __launch_bounds__(kTCThreads, 1)
       if constexpr (TT == 32) {
 #pragma unroll
         for (int k = 0; k < HPW; ++k) {
-          const int hh = sw + kSoftmaxWarps * k;
+          const int hh = softmax_head(sw, k, H_own, hbal);
 #pragma unroll
           for (int jj = 0; jj < DHB; ++jj) {
             const float4* qv = reinterpret_cast<const float4*>(q_s + (hh < H_own ? hh : 0) * DH + 8 * ((lane & 7) + 8 * jj));
             const float4 qa = qv[0], qb = qv[1];
-            qr[k][jj][0] = qa.x; qr[k][jj][1] = qa.y; qr[k][jj][2] = qa.z; qr[k][jj][3] = qa.w;
-            qr[k][jj][4] = qb.x; qr[k][jj][5] = qb.y; qr[k][jj][6] = qb.z; qr[k][jj][7] = qb.w;
+            qp[k][jj][0] = pack2(qa.x, qa.y);
+            qp[k][jj][1] = pack2(qa.z, qa.w);
+            qp[k][jj][2] = pack2(qb.x, qb.y);
+            qp[k][jj][3] = pack2(qb.z, qb.w);
           }
         }
       }
@@ -444,7 +486,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
           const int fr0 = max(nb_old - r_lo, 0);
 #pragma unroll
           for (int k = 0; k < HPW; ++k) {
-            const int hh = sw + kSoftmaxWarps * k;
+            const int hh = softmax_head(sw, k, H_own, hbal);
             if (hh >= H_own) continue;
 #pragma unroll
             for (int c = 0; c < DHB; ++c) {
@@ -480,7 +522,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
           const int c = lane & 7, rg = lane >> 3;
 #pragma unroll
           for (int k = 0; k < HPW; ++k) {
-            const int hh = sw + kSoftmaxWarps * k;
+            const int hh = softmax_head(sw, k, H_own, hbal);
             sc[k] = -INFINITY;
             if (hh >= H_own) continue;  // warp-uniform: this warp has no head in slot k
             float pr[8];
@@ -488,7 +530,8 @@ __global__ void __launch_bounds__(kTCThreads, 1)
             for (int i = 0; i < 8; ++i) {
               const int r = rg + 4 * i;
               const uint32_t rbase = kt + (r >> 4) * slab_bytes + (r & 15) * 128;
-              float a0 = 0.f, a1 = 0.f;
+              // even columns accumulate in the low half, odd columns in the high half
+              uint64_t acc = pack2(0.f, 0.f);
 #pragma unroll
               for (int jj = 0; jj < DHB; ++jj) {
                 const int colk = hh * DH + 8 * (c + 8 * jj);
@@ -496,16 +539,12 @@ __global__ void __launch_bounds__(kTCThreads, 1)
                 asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                              : "=r"(kv.x), "=r"(kv.y), "=r"(kv.z), "=r"(kv.w)
                              : "r"(rbase + (colk >> 6) * 2048 + ((((colk & 63) >> 3) ^ (r & 7)) << 4)));
-                a0 = fmaf(bf16lo(kv.x), qr[k][jj][0], a0);
-                a1 = fmaf(bf16hi(kv.x), qr[k][jj][1], a1);
-                a0 = fmaf(bf16lo(kv.y), qr[k][jj][2], a0);
-                a1 = fmaf(bf16hi(kv.y), qr[k][jj][3], a1);
-                a0 = fmaf(bf16lo(kv.z), qr[k][jj][4], a0);
-                a1 = fmaf(bf16hi(kv.z), qr[k][jj][5], a1);
-                a0 = fmaf(bf16lo(kv.w), qr[k][jj][6], a0);
-                a1 = fmaf(bf16hi(kv.w), qr[k][jj][7], a1);
+                acc = ffma2(pack2(bf16lo(kv.x), bf16hi(kv.x)), qp[k][jj][0], acc);
+                acc = ffma2(pack2(bf16lo(kv.y), bf16hi(kv.y)), qp[k][jj][1], acc);
+                acc = ffma2(pack2(bf16lo(kv.z), bf16hi(kv.z)), qp[k][jj][2], acc);
+                acc = ffma2(pack2(bf16lo(kv.w), bf16hi(kv.w)), qp[k][jj][3], acc);
               }
-              pr[i] = a0 + a1;
+              pr[i] = unpack_sum(acc);
             }
             // butterfly over the chunk lanes: after the level with mask m each lane keeps the
             // rows whose index bit (m) matches its own chunk bit, summed over both lanes
@@ -532,7 +571,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
 #pragma unroll
           for (int ps = 0; ps < NPASS; ++ps) {
             const int k = ps * HPP + hslot;
-            const int hh = sw + kSoftmaxWarps * k;
+            const int hh = softmax_head(sw, k, H_own, hbal);
             float a0 = 0.f, a1 = 0.f;
             if (k < HPW && hh < H_own) {
               const uint32_t rbase = kt + (row >> 4) * slab_bytes + (row & 15) * 128;
@@ -570,7 +609,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
 #pragma unroll
         for (int ps = 0; ps < NPASS; ++ps) {
           const int k = ps * HPP + hslot;
-          const int hh = sw + kSoftmaxWarps * k;
+          const int hh = softmax_head(sw, k, H_own, hbal);
           if (k >= HPW || hh >= H_own) continue;
           float alpha = 1.f;
           if (t == 0) {
@@ -580,7 +619,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
             mref[ps] = mx[ps];
             lsum[ps] *= alpha;
           }
-          const int m = p_row(head0 + hh, CL, H_own);
+          const int m = mrow[ps];
           const float pv = row < nvalid ? exp2f(sc[ps] - mref[ps]) : 0.f;
           const __nv_bfloat16 pb = __float2bfloat16_rn(pv);
           lsum[ps] += __bfloat162float(pb);
@@ -599,7 +638,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
           constexpr int kChunks = HPW * (TT / 8);
           if (lane < kChunks || lane >= 32 - HPW) {
             const int k = lane < kChunks ? lane / (TT / 8) : 31 - lane;
-            const int hh = sw + kSoftmaxWarps * k;
+            const int hh = softmax_head(sw, k, H_own, hbal);
             if (hh < H_own) {
               const int m = p_row(head0 + hh, CL, H_own);
               const uint32_t bar = smem_u32(&pfull[s]);
@@ -641,7 +680,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
 #pragma unroll
       for (int ps = 0; ps < NPASS; ++ps) {
         const int k = ps * HPP + hslot;
-        const int hh = sw + kSoftmaxWarps * k;
+        const int hh = softmax_head(sw, k, H_own, hbal);
         float tot = lsum[ps];
 #pragma unroll
         for (int o = TT / 2; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);

@@ -17,8 +17,9 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;
 //   meta[0]          total number of work items
 //   meta[1 + b]      first item of sequence b (b = 0..B), meta[1 + B] = total
 //   meta[2 + B + b]  flags of sequence b (kSeqAppend: lens[b] must advance by one)
+//   meta[2 + 2B]     chunk length the plan chose (the next plan's first candidate)
 constexpr int kSeqAppend = 1;
-__host__ __device__ inline size_t meta_ints(int B) { return static_cast<size_t>(2 * B + 2); }
+__host__ __device__ inline size_t meta_ints(int B) { return static_cast<size_t>(2 * B + 3); }
 
 // Scratch of the split-T orderings, carved from the caller's workspace.
 struct SplitWorkspace {

@@ -58,6 +58,10 @@ __device__ inline void plan_split(const int32_t* __restrict__ lens, int B, int64
                                   int max_items, int min_rows, int* s_nb, int* s_rows, int* s_off, int32_t* meta,
                                   int32_t* status, bool report) {
   const int lane = threadIdx.x & 31;
+  // one slot group per item (a single candidate k below): the previous plan's chunk is read with
+  // the lengths and tried first
+  const bool single_k = 2LL * n_groups > max_items || max(2 * n_groups, B) > max_items;
+  const int hint = single_k ? __ldcg(meta + 2 + 2 * B) : 0;
   int bad = 0, nonempty = 0, max_nb = 0;
   long long R = 0;
   for (int b = lane; b < B; b += 32) {
@@ -86,10 +90,29 @@ __device__ inline void plan_split(const int32_t* __restrict__ lens, int B, int64
   if (report && lane == 0 && bad) atomicOr(status, bad);
   __syncwarp();
 
+  // Fast path: the chunk the previous plan on this workspace chose is the answer again when it
+  // is still the smallest feasible one, i.e. it fits n_slots and 16 rows less does not (or is
+  // below the lower bound). Lengths usually grow by one row per step, so it rarely changes.
+  const unsigned n1 = static_cast<unsigned>(max(n_groups, nonempty));
+  const int lo16 = max((max(min_rows, 16) + 15) >> 4,
+                       static_cast<int>((static_cast<unsigned>(R) + 16u * n1 - 1u) / (16u * n1)));
+  bool fast = false;
+  if (single_k && hint >= 16 && (hint & 15) == 0 && (hint >> 4) >= lo16 && hint <= max(max_nb, 16) + 16) {
+    unsigned c0 = 0, c1 = 0;
+    const unsigned C0 = static_cast<unsigned>(hint), C1 = C0 - 16u;
+    for (int b = lane; b < B; b += 32) {
+      const unsigned nb = static_cast<unsigned>(s_nb[b]);
+      c0 += (nb + C0 - 1u) / C0;
+      if (C1 > 0u) c1 += (nb + C1 - 1u) / C1;
+    }
+    c0 = __reduce_add_sync(0xffffffffu, c0);
+    c1 = __reduce_add_sync(0xffffffffu, c1);
+    fast = c0 <= n1 && ((hint >> 4) == lo16 || c1 > n1);
+  }
   constexpr long long kItemCostRows = 128;  // epilogue + pipeline restart, in K rows
-  int chunk = 16;
-  long long best = -1;
-  for (int k = 1; static_cast<long long>(k) * n_groups <= max_items || k == 1; k <<= 1) {
+  int chunk = fast ? hint : 16;
+  long long best = fast ? 0 : -1;
+  for (int k = 1; !fast && (static_cast<long long>(k) * n_groups <= max_items || k == 1); k <<= 1) {
     const unsigned n_slots = static_cast<unsigned>(max(k * n_groups, nonempty));
     if (n_slots > static_cast<unsigned>(max_items) && k > 1) break;
     const int C = plan_chunk(s_nb, B, n_slots, min_rows, static_cast<unsigned>(R), nonempty, max_nb);
@@ -127,7 +150,10 @@ __device__ inline void plan_split(const int32_t* __restrict__ lens, int B, int64
   __syncwarp();
   if (report) {
     for (int b = lane; b <= B; b += 32) meta[1 + b] = s_off[b];
-    if (lane == 0) meta[0] = carry;
+    if (lane == 0) {
+      meta[0] = carry;
+      meta[2 + 2 * B] = chunk;
+    }
   }
 }
 
