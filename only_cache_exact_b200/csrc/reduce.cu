@@ -346,9 +346,10 @@ constexpr int kLeanThreads = 256;
 constexpr int kLeanDh = 64;
 constexpr int kLeanMaxCols = 1280;
 constexpr int kLeanCols = kLeanMaxCols / kLeanThreads;  // columns of ū per thread
+constexpr int kLeanWBlk = kLeanThreads / 32;              // items per sequence <= 32 * kLeanWBlk
 
 struct LeanSmem {
-  uint32_t w, u, ml, red, bars, total;
+  uint32_t w, u, wt, red, bars, total;
 };
 __host__ __device__ inline LeanSmem lean_smem_layout(int d, int cap_items, int max_items) {
   LeanSmem s;
@@ -357,14 +358,27 @@ __host__ __device__ inline LeanSmem lean_smem_layout(int d, int cap_items, int m
   o += up_to(static_cast<uint32_t>(d) * kLeanDh * 2u, 1024u);
   s.u = o;  // [cap_items][d] fp32
   o += static_cast<uint32_t>(cap_items) * d * 4u;
-  s.ml = o;  // m then l of the sequence's items
-  o += up_to(2u * static_cast<uint32_t>(max_items) * 4u, 16u);
+  s.wt = o;  // merge weight of every item of the sequence
+  o += up_to(static_cast<uint32_t>(max_items) * 4u, 16u);
   s.red = o;  // [8 warps][64]
   o += (kLeanThreads / 32) * kLeanDh * 4u;
   s.bars = o;
   o += 32u;
   s.total = o + 1024u;  // slack to align the base to 1024 bytes
   return s;
+}
+
+// Warp 0: U rows of head h of items lo + r0 .. (at most cap) into shared memory, one bulk copy
+// per lane, completing on ubar.
+__device__ __forceinline__ void lean_stage(float* us, const float* U, int lo, int r0, int n, int cap, int H, int h,
+                                           int d, uint64_t* ubar, int lane) {
+  const int nr = min(n - r0, cap);
+  const uint32_t row_bytes = static_cast<uint32_t>(d) * 4u;
+  if (lane == 0) mbar_arrive_expect_tx(ubar, static_cast<uint32_t>(nr) * row_bytes);
+  __syncwarp();
+  for (int c = lane; c < nr; c += 32)
+    bulk_load_g2s(us + static_cast<size_t>(c) * d, U + (static_cast<size_t>(lo + r0 + c) * H + h) * d, row_bytes,
+                  ubar);
 }
 
 __global__ void __launch_bounds__(kLeanThreads, 1)
@@ -375,9 +389,8 @@ __global__ void __launch_bounds__(kLeanThreads, 1)
   const int h = blockIdx.x, b = blockIdx.y, d = p.d;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   float* us = reinterpret_cast<float*>(sm + L.u);
-  float* ms = reinterpret_cast<float*>(sm + L.ml);
-  float* ls = ms + p.max_items;
   float* red = reinterpret_cast<float*>(sm + L.red);
+  float* ws_ = reinterpret_cast<float*>(sm + L.wt);
   uint64_t* wbar = reinterpret_cast<uint64_t*>(sm + L.bars);
   uint64_t* ubar = wbar + 1;
   int* rng = reinterpret_cast<int*>(wbar + 2);
@@ -399,27 +412,35 @@ __global__ void __launch_bounds__(kLeanThreads, 1)
   if (h == 0 && tid == 32 && (__ldcg(p.meta + 2 + p.B + b) & kSeqAppend)) p.lens[b] += 1;
   __syncthreads();
   const int lo = rng[0], n = rng[1] - lo;
-  const uint32_t row_bytes = static_cast<uint32_t>(d) * 4u;
-  auto stage = [&](int r0) {  // one thread: U rows of items lo + r0 .. into shared memory
-    const int nr = min(n - r0, p.cap_items);
-    mbar_arrive_expect_tx(ubar, static_cast<uint32_t>(nr) * row_bytes);
-    for (int c = 0; c < nr; ++c)
-      bulk_load_g2s(us + static_cast<size_t>(c) * d, p.U + (static_cast<size_t>(lo + r0 + c) * p.H + h) * d,
-                    row_bytes, ubar);
-  };
-  if (tid == 0 && n > 0) stage(0);
-  for (int c = tid; c < n; c += kLeanThreads) {
-    ms[c] = __ldcg(p.m + static_cast<size_t>(lo + c) * p.H + h);
-    ls[c] = __ldcg(p.l + static_cast<size_t>(lo + c) * p.H + h);
-  }
-  __syncthreads();
+  if (warp == 0 && n > 0) lean_stage(us, p.U, lo, 0, n, p.cap_items, p.H, h, d, ubar, lane);
 
-  // merge weights, computed by every thread from the shared m, l
-  float M = -INFINITY;
-  for (int c = 0; c < n; ++c) M = fmaxf(M, ms[c]);
+  // merge weights 2^(m_c - M) / Σ_c' 2^(m_c' - M) l_c': every warp loads every item's m and l at
+  // once (lane c % 32 of block c / 32) and finds M and the sum itself, so no barrier separates
+  // them; warp j writes the weights of block j, published by the barrier of the first U wait
+  const float* mh = p.m + static_cast<size_t>(lo) * p.H + h;
+  const float* lh = p.l + static_cast<size_t>(lo) * p.H + h;
+  float mv[kLeanWBlk], lv[kLeanWBlk];
+#pragma unroll
+  for (int j = 0; j < kLeanWBlk; ++j) {
+    const int c = lane + 32 * j;
+    mv[j] = c < n ? mh[static_cast<size_t>(c) * p.H] : -INFINITY;
+    lv[j] = c < n ? lh[static_cast<size_t>(c) * p.H] : 0.f;
+  }
+  float M = mv[0];
+#pragma unroll
+  for (int j = 1; j < kLeanWBlk; ++j) M = fmaxf(M, mv[j]);
+  M = warp_max(M);
   float S = 0.f;
-  for (int c = 0; c < n; ++c) S = fmaf(exp2f(ms[c] - M), ls[c], S);
+#pragma unroll
+  for (int j = 0; j < kLeanWBlk; ++j) {
+    mv[j] = lane + 32 * j < n ? exp2f(mv[j] - M) : 0.f;
+    S = fmaf(mv[j], lv[j], S);
+  }
+  S = warp_sum(S);
   const float inv = S > 0.f ? 1.f / S : 0.f;
+#pragma unroll
+  for (int j = 0; j < kLeanWBlk; ++j)
+    if (warp == j && lane + 32 * j < n) ws_[lane + 32 * j] = mv[j] * inv;
 
   float ub[kLeanCols];
 #pragma unroll
@@ -431,7 +452,7 @@ __global__ void __launch_bounds__(kLeanThreads, 1)
     if (!ok) break;
     const int nr = min(n - r0, p.cap_items);
     for (int c = 0; c < nr; ++c) {
-      const float w = exp2f(ms[r0 + c] - M) * inv;
+      const float w = ws_[r0 + c];
       const float* row = us + static_cast<size_t>(c) * d;
 #pragma unroll
       for (int i = 0; i < kLeanCols; ++i) {
@@ -441,7 +462,7 @@ __global__ void __launch_bounds__(kLeanThreads, 1)
     }
     if (r0 + p.cap_items < n) {
       __syncthreads();  // every thread is done with the staged rows
-      if (tid == 0) stage(r0 + p.cap_items);
+      if (warp == 0) lean_stage(us, p.U, lo, r0 + p.cap_items, n, p.cap_items, p.H, h, d, ubar, lane);
     }
   }
   ok = __syncthreads_and(ok && mbar_wait(wbar, 0u, p.status));
@@ -582,6 +603,7 @@ namespace {
 int lean_cap_items(int B, int d, int H, int dtype, int max_items) {
   if (dtype != SLIM_BF16 || H * kLeanDh != d || d % kLeanThreads || d > kLeanMaxCols) return 0;
   if (static_cast<long long>(B) * H > num_sms()) return 0;  // one wave (one CTA per SM)
+  if (max_items > 32 * kLeanWBlk) return 0;                  // items' merge weights: one per thread
   const int optin = max_smem_optin();
   const uint32_t fixed = lean_smem_layout(d, 0, max_items).total;
   if (fixed >= static_cast<uint32_t>(optin)) return 0;
