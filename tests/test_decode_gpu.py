@@ -57,6 +57,15 @@ def test_cross_attention_fixed_cache_d1280(S):
     assert torch.equal(g.lens.cpu(), torch.from_numpy(c.lens))
 
 
+def test_long_single_sequence_merged_in_rounds(S):
+    # One 6000-row sequence at d=1024 is cut into ~47 work items, more than the one-sequence
+    # merge stages in shared memory at once, so its U rows arrive in several rounds.
+    c = make_case(1024, 16, lens=[6000], cap=6100, seed=12)
+    g = GpuState(c, S)
+    _check_bf16(g.step(S.SLIM_VARIANT_B), oracle_out(c), c.H)
+    assert int(g.status.item()) == 0
+
+
 def test_d4096_four_cta_cluster(S):
     c = make_case(4096, 32, lens=[700, 333, 64], cap=800, seed=3)
     g = GpuState(c, S)
