@@ -1,23 +1,33 @@
 """Benchmark of the Slim attention decode step (K-only cache) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+                    [--no-extras]
 
 One step = one slim_decode_step over the whole batch: append this step's k,
 scores of q against the K cache, softmax, V = K·W_KV by the selected
-ordering, output. The default workload is d=1024, H=16 (d_h=64), B=8, a
-4096-token bf16 K cache per sequence with fp32 accumulation. Inputs are seeded
-synthetic data (X ~ N(0,1), W_K = orthogonal·diag(U[0.5,2]), W_V ~ N(0,1/d)),
-generated by only_cache_exact_b200.synth; the K cache is filled by the
-library's own prompt-phase kernel.
+ordering, output. The headline workload is the largest one that fits one GPU:
+7B-style MHA decode, d=4096, H=32 (d_h=128), B=16 sequences with ragged
+cached lengths uniform in [16384, 32768], bf16 K cache, fp32 accumulation.
+Inputs are seeded synthetic data (X ~ N(0,1), W_K = orthogonal·diag(U[0.5,2]),
+W_V ~ N(0,1/d)) from only_cache_exact_b200.synth; the K cache is filled by the
+library's own prompt-phase kernel from prompt rows drawn on the device.
 
-Timing: W untimed warm-up steps, then exactly K steps replayed from CUDA
-graphs, bracketed by a barrier and a device synchronise, timed with CUDA
-events on the launching stream; the max over ranks is reported. Enough
-copies of the cache, W_KV and step inputs are rotated to exceed twice the
-126 MB L2, so every step reads its K cache from HBM. Lengths are reset to T
-before each measured region; each step appends one row, so the attended
-length grows by one per step of the same buffer set and the byte counts
-follow the actual lengths.
+Timing: W untimed warm-up steps and one untimed replay of every captured CUDA
+graph, then exactly K steps replayed from CUDA graphs, bracketed by a barrier
+and a device synchronise, timed with CUDA events on the launching stream; the
+max over ranks is reported. Between steps either the K cache alone exceeds
+twice the 126 MB L2, or enough copies of the cache, W_KV and the step inputs
+rotate to exceed it, or (tiny workloads) a 256 MB buffer is written before
+each step, which is then timed alone; `config.l2` says which. Lengths are reset
+before each measured region; each step appends one row, so the attended length
+grows by one per step of the same buffer set and the byte counts follow the
+actual lengths.
+
+With one GPU the same line also carries one record per other workload
+(`workloads`), each with its own step count, roofline and oracle baseline;
+the ordering (a)/(b) sweep over T = 1K..128K at d=4096, H=32, B=1
+(`sweep`); the prompt-phase projection (`prefill`); and ordering (a) on the
+d=1024 workload (`variant_a`).
 
 Multi-GPU: sequences are independent, so every rank runs its own batch
 (weak scaling, no collective on the data path); value = all ranks' steps /
@@ -33,7 +43,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -46,32 +55,41 @@ sys.path.insert(0, ROOT)
 METRIC = "slim decode steps/s and achieved HBM GB/s vs B200 peak (K-only cache)"
 
 WORKLOADS = {
-    # name: d, H, B, T (cached rows before the first step), dtype, append
-    "d1024_h16_b8_t4096": dict(d=1024, H=16, B=8, T=4096, dtype="bf16", append=True,
+    # name: d, H, B, T (cached rows before the first step), dtype, append, steps (sub-record step count)
+    "d4096_h32_b16_t16k_32k": dict(d=4096, H=32, B=16, T=(16384, 32768), dtype="bf16", append=True, steps=20,
+                                   desc="7B-style MHA decode, d=4096 H=32 d_h=128, B=16, ragged T in [16K,32K], "
+                                        "bf16 K cache, fp32 accumulation"),
+    "d256_h4_b1_t128_f32": dict(d=256, H=4, B=1, T=128, dtype="f32", append=True, steps=16,
+                                desc="single MHA layer fp32, d=256 H=4 d_h=64, B=1, 128-token prompt then "
+                                     "16 decode steps"),
+    "d1024_h16_b8_t4096": dict(d=1024, H=16, B=8, T=4096, dtype="bf16", append=True, steps=64,
                                desc="decode step, d=1024 H=16 d_h=64, B=8, T=4096 bf16 K cache, fp32 accumulation"),
-    "d4096_h32_b16_t16k_32k": dict(d=4096, H=32, B=16, T=(16384, 32768), dtype="bf16", append=True,
-                                   desc="7B-style MHA decode, d=4096 H=32 d_h=128, B=16, ragged T in [16K,32K]"),
-    "d1280_h20_b64_t1500_cross": dict(d=1280, H=20, B=64, T=1500, dtype="bf16", append=False,
-                                      desc="cross-attention decode, d=1280 H=20, B=64, fixed 1500-row K cache"),
-    "d4096_h32_b1_t131072": dict(d=4096, H=32, B=1, T=131072 - 64 * 64, dtype="bf16", append=True,
-                                 desc="long-context decode, d=4096 H=32, B=1, T~128K"),
+    "d1280_h20_b64_t1500_cross": dict(d=1280, H=20, B=64, T=1500, dtype="bf16", append=False, steps=448,
+                                      desc="encoder-decoder cross-attention decode, d=1280 H=20 d_h=64, B=64, "
+                                           "fixed 1500-row encoder K cache, 448 steps"),
+    "d4096_h32_b1_t8192": dict(d=4096, H=32, B=1, T=8192, dtype="bf16", append=True, steps=64,
+                               desc="long-context layer, d=4096 H=32, B=1: 64 decode steps after the "
+                                    "8192-token prompt"),
+    "d4096_h32_b1_t131072": dict(d=4096, H=32, B=1, T=131072 - 80, cap=131072, dtype="bf16", append=True,
+                                 steps=64, desc="long-context decode, d=4096 H=32, B=1, 64 steps at the end of "
+                                                "the 131072-row K cache"),
 }
-DEFAULT = "d1024_h16_b8_t4096"
+DEFAULT = "d4096_h32_b16_t16k_32k"
+SUBRECORDS = ["d256_h4_b1_t128_f32", "d1024_h16_b8_t4096", "d1280_h20_b64_t1500_cross", "d4096_h32_b1_t8192",
+              "d4096_h32_b1_t131072"]
+FLUSH_BYTES = 256 << 20
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT, choices=sorted(WORKLOADS))
-    ap.add_argument("--rot", type=int, default=0, help="buffer sets rotated (0: enough for 2x L2)")
-    ap.add_argument("--no-extras", action="store_true", help="skip the ordering-(a), prefill and CPU legs")
+    ap.add_argument("--rot", type=int, default=0, help="buffer sets rotated (0: automatic)")
+    ap.add_argument("--no-extras", action="store_true", help="headline line only (no sub-records, sweep, CPU legs)")
     ap.add_argument("--ref-seconds", type=float, default=20.0, help="CPU time budget of --impl reference")
-    ap.add_argument("--sweep", action="store_true",
-                    help="ordering (a) vs (b) crossover over T=1K..128K at d=4096 H=32 B=1 (one JSON line per T), "
-                         "and the 8192-token prompt projection; not part of the default run")
     return ap.parse_args()
 
 
@@ -128,7 +146,7 @@ class ClockSampler:
     def _run(self):
         while not self._stop.is_set():
             self.sample()
-            time.sleep(0.01)
+            time.sleep(0.005)
 
     def sample(self):
         if self.nv is None:
@@ -155,23 +173,26 @@ class ClockSampler:
                 "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
-def profile_traffic(name):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged since."""
-    path = os.path.join(ROOT, "profiles", name)
-    src = os.path.join(ROOT, "only_cache_exact_b200", "csrc", "decode_b_tc.cu")
+def kernel_sources_sha():
+    """Hash of the split kernel's sources; a stored ncu figure is used only while it matches."""
+    h = hashlib.sha256()
+    for f in ("decode_b_tc.cu", "split_plan.cuh", "ptx.cuh"):
+        h.update(open(os.path.join(ROOT, "only_cache_exact_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(workload):
+    """DRAM bytes per split-kernel launch from profiles/decode_b_tc_<workload>.json (an ncu capture),
+    if the kernel sources are unchanged since it was taken; else None."""
+    path = os.path.join(ROOT, "profiles", f"decode_b_tc_{workload}.json")
     if not os.path.exists(path):
         return None
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    kv = {}
-    for line in open(path):
-        if ":" in line and line.startswith("- "):
-            k, v = line[2:].split(":", 1)
-            kv[k.strip()] = v.strip().strip("`")
-    if kv.get("source_sha256_16") != sha:
-        return None
     try:
-        return float(kv["dram_bytes_per_launch"])
-    except (KeyError, ValueError):
+        j = json.load(open(path))
+        if j.get("source_sha256_16") != kernel_sources_sha():
+            return None
+        return float(j["dram_bytes_per_launch"])
+    except (ValueError, KeyError, OSError):
         return None
 
 
@@ -183,245 +204,317 @@ def peaks():
     return 6650.0, 1590.0, "fallback"
 
 
-# ------------------------------------------------------------------------------------------ our arm
-def run_ours(args, rank, world, local, pg):
-    import torch
+def cpu_oracle_rate(w, budget_s=12.0):
+    """Oracle step time on the host: float64 standard MHA with explicit K and V caches, one sequence
+    at a time (sequences are independent), as many steps as fit in the budget, scaled to the batch."""
+    from threadpoolctl import threadpool_info
 
-    from only_cache_exact_b200 import params, replicas, slim as S, synth
+    from oracle import slim_oracle as O
+    d, H = w["d"], w["H"]
+    lens = seq_lengths(w)
+    T = int(np.max(lens)) + (1 if w["append"] else 0)
+    rng = np.random.default_rng(0)
+    K = rng.standard_normal((T, d))
+    V = rng.standard_normal((T, d))
+    q = rng.standard_normal(d)
+    O.mha_decode(q, K, V, H)  # warm
+    n, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < budget_s or n == 0:
+        O.mha_decode(q, K, V, H)
+        n += 1
+    per_seq = (time.perf_counter() - t0) / n
+    # one step = every sequence of the batch (ragged: scaled by the attended rows)
+    step_s = per_seq * float(np.sum(lens + (1 if w["append"] else 0))) / T
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return 1.0 / step_s, threads, n, T
 
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    w = WORKLOADS[args.workload]
-    d, H, B = w["d"], w["H"], w["B"]
-    lens0 = seq_lengths(w)
-    gids = replicas.global_sequence_ids(rank, world, B)  # this rank's own token streams
-    append = w["append"]
-    K_steps, W_steps = args.steps, args.warmup
-    tdt = torch.bfloat16 if w["dtype"] == "bf16" else torch.float32
-    dt_code = S.SLIM_BF16 if w["dtype"] == "bf16" else S.SLIM_F32
-    esz = 2 if w["dtype"] == "bf16" else 4
-    cache_bytes_one = int(B * int(lens0.max()) * d * esz)
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    rot = args.rot or max(1, min(8, -(-2 * l2 // max(cache_bytes_one, 1)) + 1))
-    if cache_bytes_one * rot > 100e9:
-        rot = 1
-    G = max(rot, min(K_steps, 256) // rot * rot)
-    e2e_steps = max(8, min(K_steps, 200))
-    # appended rows per buffer set between two length resets (the largest measured region)
-    per_set_appends = -(-max(K_steps, W_steps, G, e2e_steps + 3, 32) // rot) if append else 0
-    cap = int(lens0.max()) + per_set_appends + 8
 
-    wts = synth.make_weights(d, 0, w["dtype"])
-    W_K = synth.to_storage(wts.W_K, w["dtype"]).to(dev)
-    W_KV0 = params.make_wkv(wts.W_K, wts.W_V, dtype=tdt, device=dev)
-    status = torch.zeros(1, dtype=torch.int32, device=dev)
-    # cache of buffer set 0 filled by the prompt-phase kernel, sequence by sequence
-    K0 = torch.zeros(B, cap, d, dtype=tdt, device=dev)
-    lens_dev0 = torch.zeros(B, dtype=torch.int32, device=dev)
-    t_fill = time.perf_counter()
-    for b in range(B):
-        n = int(lens0[b])
-        for r0 in range(0, n, 8192):
-            r1 = min(n, r0 + 8192)
-            Xb = synth.to_storage(synth.make_tokens(r1 - r0, d, 1000 + r0, gids[b], w["dtype"]), w["dtype"]).to(dev)
-            S.slim_prefill_k(Xb.view(1, r1 - r0, d), W_K, K0[b:b + 1], lens_dev0[b:b + 1], status)
-    torch.cuda.synchronize()
-    t_fill = time.perf_counter() - t_fill
-    x_new = np.stack([synth.make_tokens(1, d, 0, gids[b], w["dtype"], part=2)[0] for b in range(B)])
-    q0 = torch.from_numpy(x_new @ wts.W_Q).float().to(dev)
-    k0 = synth.to_storage(synth.round_to(x_new @ wts.W_K, w["dtype"]), w["dtype"]).to(dev) if append else None
+# ------------------------------------------------------------------------------------------ one workload
+class Workload:
+    """Device state of one workload: K cache(s) filled by the prompt-phase kernel, W_KV, step inputs."""
 
-    sets = []
-    for i in range(rot):
-        sets.append(dict(K=K0 if i == 0 else K0.clone(), lens=lens_dev0.clone(), W_KV=W_KV0.clone(),
-                         q=q0.clone(), k=None if k0 is None else k0.clone(),
-                         out=torch.empty(B, d, dtype=torch.float32, device=dev),
-                         ws=S.alloc_workspace(dt_code, B, d, H, cap, S.SLIM_AUTO, device=dev)))
-    torch.cuda.synchronize()
-    t_hint = int(lens0.max())
+    def __init__(self, name, S, dev, rank=0, world=1, max_steps=256, rot=0):
+        import torch
 
-    def step(i, variant=S.SLIM_AUTO):
-        s = sets[i % rot]
-        S.slim_decode_step(s["q"], s["k"], s["K"], s["lens"], s["W_KV"], H, s["out"], s["ws"], status,
-                           variant=variant, t_hint=t_hint)
-
-    stream = torch.cuda.Stream(device=dev)
-    torch.cuda.synchronize()
-
-    # warm-up (eager), also resolves the ordering
-    with torch.cuda.stream(stream):
-        for i in range(W_steps):
-            step(i)
-    stream.synchronize()
-    chosen = S.slim_select_variant(dt_code, B, d, H, t_hint)
-    launches_per_step = S.slim_last_launch_count()
-
-    def reset_lengths():
-        for st_ in sets:
-            st_["lens"].copy_(lens_dev0)
+        from only_cache_exact_b200 import params, replicas, synth
+        self.name, self.S, self.dev = name, S, dev
+        w = self.w = WORKLOADS[name]
+        d, H, B = w["d"], w["H"], w["B"]
+        self.d, self.H, self.B = d, H, B
+        self.append = w["append"]
+        self.lens0 = seq_lengths(w)
+        gids = replicas.global_sequence_ids(rank, world, B)  # this rank's own token streams
+        self.tdt = torch.bfloat16 if w["dtype"] == "bf16" else torch.float32
+        self.dt_code = S.SLIM_BF16 if w["dtype"] == "bf16" else S.SLIM_F32
+        self.esz = 2 if w["dtype"] == "bf16" else 4
+        set_bytes = int(np.sum(self.lens0)) * d * self.esz + d * d * self.esz
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        if rot:
+            self.rot = rot
+        elif set_bytes >= 2 * l2:
+            self.rot = 1
+        else:
+            self.rot = min(8, -(-2 * l2 // set_bytes) + 1)
+        self.flush = self.rot * set_bytes < 2 * l2  # too small to rotate past L2: flush before each step
+        if self.flush:
+            self.rot = 1
+        per_set_appends = -(-max_steps // self.rot) + 4 if self.append else 0
+        self.cap = int(np.max(self.lens0)) + per_set_appends + 8
+        if "cap" in w:
+            self.cap = min(self.cap, int(w["cap"]))
+            if self.append and self.cap < int(np.max(self.lens0)) + -(-max_steps // self.rot):
+                raise ValueError(f"{name}: {max_steps} steps do not fit the {self.cap}-row cache")
+        wts = synth.make_weights(d, 0, w["dtype"])
+        self.W_K = synth.to_storage(wts.W_K, w["dtype"]).to(dev)
+        W_KV0 = params.make_wkv(wts.W_K, wts.W_V, dtype=self.tdt, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        K0 = torch.zeros(B, self.cap, d, dtype=self.tdt, device=dev)
+        lens_dev0 = torch.zeros(B, dtype=torch.int32, device=dev)
+        t = time.perf_counter()
+        for b in range(B):
+            n = int(self.lens0[b])
+            for r0 in range(0, n, 8192):
+                r1 = min(n, r0 + 8192)
+                Xb = synth.make_tokens_device(r1 - r0, d, 1000 + r0 // 8192, gids[b], w["dtype"], device=dev)
+                S.slim_prefill_k(Xb.view(1, r1 - r0, d), self.W_K, K0[b:b + 1], lens_dev0[b:b + 1], self.status)
+        torch.cuda.synchronize()
+        self.fill_s = time.perf_counter() - t
+        self.lens_dev0 = lens_dev0
+        x_new = np.stack([synth.make_tokens(1, d, 0, gids[b], w["dtype"], part=2)[0] for b in range(B)])
+        self.q0 = torch.from_numpy(x_new @ wts.W_Q).float().to(dev)
+        self.k0 = (synth.to_storage(synth.round_to(x_new @ wts.W_K, w["dtype"]), w["dtype"]).to(dev)
+                   if self.append else None)
+        self.sets = []
+        for i in range(self.rot):
+            self.sets.append(dict(K=K0 if i == 0 else K0.clone(), lens=lens_dev0.clone(),
+                                  W_KV=W_KV0 if i == 0 else W_KV0.clone(),
+                                  q=self.q0.clone(), k=None if self.k0 is None else self.k0.clone(),
+                                  out=torch.empty(B, d, dtype=torch.float32, device=dev),
+                                  ws=S.alloc_workspace(self.dt_code, B, d, H, self.cap, S.SLIM_AUTO, device=dev)))
+        self.t_hint = int(np.max(self.lens0))
+        self.stream = torch.cuda.Stream(device=dev)
+        self.flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev) if self.flush else None
         torch.cuda.synchronize()
 
-    def rows_attended(nsteps):
+    def step(self, i, variant=None):
+        S = self.S
+        s = self.sets[i % self.rot]
+        S.slim_decode_step(s["q"], s["k"], s["K"], s["lens"], s["W_KV"], self.H, s["out"], s["ws"], self.status,
+                           variant=S.SLIM_AUTO if variant is None else variant, t_hint=self.t_hint)
+
+    def reset_lengths(self):
+        import torch
+        for st_ in self.sets:
+            st_["lens"].copy_(self.lens_dev0)
+        torch.cuda.synchronize()
+
+    def rows_attended(self, nsteps):
         """Rows all sequences attend over in nsteps steps started from freshly reset lengths."""
-        tot = 0
-        for s_ in range(nsteps):
-            tot += int(lens0.astype(np.int64).sum()) + B * ((s_ // rot) + 1 if append else 0)
-        return tot
+        base = int(self.lens0.astype(np.int64).sum())
+        return sum(base + (self.B * ((s_ // self.rot) + 1) if self.append else 0) for s_ in range(nsteps))
 
-    # graphs of G steps (G a multiple of the rotation) replayed to cover exactly K steps
+    def algorithmic_bytes(self, nsteps):
+        """(split kernel bytes per launch, step bytes) averaged over nsteps steps: K rows attended
+        (incl. the appended one) read once, q, k_new read and written; the step adds W_KV once and
+        the output."""
+        per_step_const = self.B * self.d * 4 + (2 * self.B * self.d * self.esz if self.append else 0)
+        kernel = self.rows_attended(nsteps) * self.d * self.esz / nsteps + per_step_const
+        return kernel, kernel + self.d * self.d * self.esz + self.B * self.d * 4
 
-    def capture(nsteps, base):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for j in range(nsteps):
-                step(base + j)
-        return g
-
-    full, rem = divmod(K_steps, G)
-    g_full = capture(G, 0) if full else None
-    g_rem = capture(rem, 0) if rem else None
-    torch.cuda.synchronize()
-
-    def run_timed():
+    def time_steps(self, K_steps, W_steps, pg=None, sample_clocks=None):
+        """Device time of exactly K_steps steps after W_steps warm-up steps (ms)."""
+        import torch
+        stream = self.stream
         with torch.cuda.stream(stream):
-            for _ in range(full):
-                g_full.replay()
-            if g_rem is not None:
-                g_rem.replay()
-
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    reset_lengths()
-    if pg:
-        pg.barrier()
-    torch.cuda.synchronize()
-    sampler = ClockSampler(local)
-    with sampler:
-        ev0.record(stream)
-        run_timed()
-        ev1.record(stream)
-        ev1.synchronize()
-    ms = ev0.elapsed_time(ev1)
-    torch.cuda.synchronize()
-    ms = replicas.max_over_ranks(ms, pg, dev)
-    st = int(status.item())
-    ms_step = ms / K_steps
-
-    # the dominant kernel (split kernel that streams the K cache), timed live with events
-    # (eager launches behind a spin kernel, so the host has enqueued every step before the GPU
-    # reaches them and consecutive launches run back to back)
-    reset_lengths()
-    S.slim_timing_enable(G)
-    with torch.cuda.stream(stream):
-        torch.cuda._sleep(int(100e6))
-        for j in range(G):
-            step(j)
-    stream.synchronize()
-    split_ms = S.slim_timing_read(G)
-    S.slim_timing_enable(0)
-    split_avg_ms = float(np.mean(split_ms)) if split_ms else None
-
-    lens_now = sets[0]["lens"].cpu().numpy()
-    # algorithmic bytes of the split kernel: K rows attended (incl. appended), q, k_new (read + write);
-    # of the step: plus W_KV once and the output
-    per_step_const = B * d * 4 + (2 * B * d * esz if append else 0)
-    kernel_bytes = rows_attended(G) * d * esz / G + per_step_const
-    step_bytes = rows_attended(K_steps) * d * esz / K_steps + per_step_const + d * d * esz + B * d * 4
-    hbm_peak, tc_peak, peak_src = peaks()
-    achieved = kernel_bytes / (split_avg_ms * 1e-3) / 1e9 if split_avg_ms else None
-
-    # end to end through the host-buffer entry point: pinned q/k in, out back, every step
-    q_h = q0.cpu().pin_memory()
-    k_h = k0.cpu().pin_memory() if k0 is not None else None
-    out_h = torch.empty(B, d, dtype=torch.float32).pin_memory()
-    reset_lengths()
-
-    def host_step(i):
-        s = sets[i % rot]
-        S.slim_decode_step_host(q_h, k_h, s["K"], s["lens"], s["W_KV"], H, out_h, s["ws"], status,
-                                variant=S.SLIM_AUTO, t_hint=t_hint, stream=stream)
-
-    for i in range(3):
-        host_step(i)
-    stream.synchronize()
-    if pg:
-        pg.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(e2e_steps):
-        host_step(i)
-    e1.record(stream)
-    e1.synchronize()
-    e2e_ms = replicas.max_over_ranks(e0.elapsed_time(e1) / e2e_steps, pg, dev)
-    assert np.all(np.isfinite(out_h.numpy()))
-
-    extras = {}
-    reset_lengths()
-    if not args.no_extras and rank == 0:
-        extras = run_extras(args, w, sets, step, stream, S, dt_code, B, d, H, K0, W_K, t_hint, rot)
-
-    res = dict(ms=ms, ms_step=ms_step, st=st, chosen=chosen, launches=launches_per_step, rot=rot, cap=cap,
-               split_avg_ms=split_avg_ms, kernel_bytes=int(kernel_bytes), step_bytes=int(step_bytes),
-               achieved=achieved, hbm_peak=hbm_peak, peak_src=peak_src, e2e_ms=e2e_ms, clocks=sampler.summary(),
-               lens_now=lens_now.tolist()[:4], extras=extras, fill_s=t_fill, G=G,
-               t_range=[int(lens0.min()), int(lens0.max()) + (-(-K_steps // rot) if append else 0)],
-               h2d=int(B * d * 4 + (B * d * esz if append else 0)), d2h=int(B * d * 4), esz=esz)
-    return res
-
-
-def run_extras(args, w, sets, step, stream, S, dt_code, B, d, H, K0, W_K, t_hint, rot):
-    """Ordering (a) on the same workload, and the prompt-phase projection of the whole cache."""
-    import torch
-    out = {}
-    if w["B"] * w["d"] <= 8 * 1024:  # (a) materialises V for the whole batch; only on the small workload
-        n = 20
-        for i in range(3):
-            step(i, S.SLIM_VARIANT_A)
+            for i in range(W_steps):
+                self.step(i)
         stream.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if self.flush:
+            # tiny workload: every step runs after a write of 256 MB, timed alone
+            self.reset_lengths()
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(K_steps)]
+            if pg:
+                pg.barrier()
+            torch.cuda.synchronize()
+            with sample_clocks or _Null():
+                with torch.cuda.stream(stream):
+                    for i in range(K_steps):
+                        self.flush_buf.fill_(i & 0xFF)
+                        evs[i][0].record(stream)
+                        self.step(i)
+                        evs[i][1].record(stream)
+                stream.synchronize()
+            return sum(a.elapsed_time(b) for a, b in evs)
+        G = max(self.rot, min(K_steps, 256) // self.rot * self.rot)
+        full, rem = divmod(K_steps, G)
+
+        def capture(nsteps):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for j in range(nsteps):
+                    self.step(j)
+            return g
+
+        g_full = capture(G) if full else None
+        g_rem = capture(rem) if rem else None
+        torch.cuda.synchronize()
+        # one untimed replay of each graph (uploads it), then back to the starting lengths
+        self.reset_lengths()
         with torch.cuda.stream(stream):
-            e0.record(stream)
-            for i in range(n):
-                step(i, S.SLIM_VARIANT_A)
-            e1.record(stream)
+            for g in (g_full, g_rem):
+                if g is not None:
+                    g.replay()
+        stream.synchronize()
+        self.reset_lengths()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize()
+        with sample_clocks or _Null():
+            ev0.record(stream)
+            with torch.cuda.stream(stream):
+                for _ in range(full):
+                    g_full.replay()
+                if g_rem is not None:
+                    g_rem.replay()
+            ev1.record(stream)
+            ev1.synchronize()
+        ms = ev0.elapsed_time(ev1)
+        del g_full, g_rem
+        return ms
+
+    def split_kernel_ms(self, n):
+        """Average duration of the split kernel (the one that streams the K cache) over n steps, from
+        event pairs the library records around it on its stream; steps queued behind a spin kernel so
+        the GPU never waits for the host."""
+        import torch
+        S = self.S
+        self.reset_lengths()
+        S.slim_timing_enable(n)
+        with torch.cuda.stream(self.stream):
+            torch.cuda._sleep(int(50e6))
+            for j in range(n):
+                if self.flush:
+                    self.flush_buf.fill_(j & 0xFF)
+                self.step(j)
+        self.stream.synchronize()
+        ms = S.slim_timing_read(n)
+        S.slim_timing_enable(0)
+        return float(np.mean(ms)) if ms else None
+
+    def e2e_ms(self, nsteps, pg=None):
+        """Per-step time through slim_decode_step_host: pinned q, k in and out back every step."""
+        import torch
+
+        from only_cache_exact_b200 import replicas
+        S = self.S
+        q_h = self.q0.cpu().pin_memory()
+        k_h = self.k0.cpu().pin_memory() if self.k0 is not None else None
+        out_h = torch.empty(self.B, self.d, dtype=torch.float32).pin_memory()
+        self.reset_lengths()
+
+        def host_step(i):
+            s = self.sets[i % self.rot]
+            S.slim_decode_step_host(q_h, k_h, s["K"], s["lens"], s["W_KV"], self.H, out_h, s["ws"], self.status,
+                                    variant=S.SLIM_AUTO, t_hint=self.t_hint, stream=self.stream)
+
+        for i in range(3):
+            host_step(i)
+        self.stream.synchronize()
+        self.reset_lengths()
+        if pg:
+            pg.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(self.stream)
+        for i in range(nsteps):
+            host_step(i)
+        e1.record(self.stream)
         e1.synchronize()
-        ms_a = e0.elapsed_time(e1) / n
-        out["variant_a"] = {"ms_per_step": round(ms_a, 5), "steps_per_s": round(1e3 / ms_a, 1)}
-    # prompt-phase projection of B sequences x 4096 rows (K = X·W_K)
-    n_rows = 4096
-    tdt = K0.dtype
-    X = torch.randn(B, n_rows, d, device=K0.device).to(tdt)
-    Kp = torch.empty(B, n_rows + 8, d, dtype=tdt, device=K0.device)
-    lens = torch.zeros(B, dtype=torch.int32, device=K0.device)
-    status = torch.zeros(1, dtype=torch.int32, device=K0.device)
-    reps = 5
-    for _ in range(2):
-        lens.zero_()
-        S.slim_prefill_k(X, W_K, Kp, lens, status)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    tot = 0.0
-    for _ in range(reps):
-        lens.zero_()
-        e0.record()
-        S.slim_prefill_k(X, W_K, Kp, lens, status)
-        e1.record()
-        e1.synchronize()
-        tot += e0.elapsed_time(e1)
-    ms_p = tot / reps
-    flops = 2.0 * B * n_rows * d * d
-    out["prefill"] = {"rows": int(B * n_rows), "ms": round(ms_p, 4), "tflops": round(flops / ms_p / 1e9, 1)}
-    return out
+        assert np.all(np.isfinite(out_h.numpy()))
+        return replicas.max_over_ranks(e0.elapsed_time(e1) / nsteps, pg, self.dev)
+
+    def measure(self, K_steps, W_steps, pg=None, clocks=None, e2e=True):
+        """Steps/s, roofline of the split kernel, e2e and footprint for this workload."""
+        from only_cache_exact_b200 import replicas
+        S = self.S
+        ms = self.time_steps(K_steps, W_steps, pg, clocks)
+        ms = replicas.max_over_ranks(ms, pg, self.dev)
+        st = int(self.status.item())
+        ms_step = ms / K_steps
+        chosen = S.slim_select_variant(self.dt_code, self.B, self.d, self.H, self.t_hint)
+        launches = S.slim_last_launch_count()
+        n_live = min(max(K_steps, 8), 64)
+        split_ms = self.split_kernel_ms(n_live)
+        kbytes, sbytes_live = self.algorithmic_bytes(n_live)
+        _, sbytes = self.algorithmic_bytes(K_steps)
+        hbm_peak, _, peak_src = peaks()
+        achieved = kbytes / (split_ms * 1e-3) / 1e9 if split_ms else None
+        r = dict(ms_step=ms_step, status=st, chosen=chosen, launches=launches, split_ms=split_ms,
+                 kernel_bytes=int(kbytes), step_bytes=int(sbytes), achieved=achieved, hbm_peak=hbm_peak,
+                 peak_src=peak_src)
+        r["e2e_ms"] = self.e2e_ms(max(8, min(K_steps, 200)), pg) if e2e else None
+        return r
+
+    def l2_note(self):
+        if self.flush:
+            return f"a {FLUSH_BYTES >> 20} MB buffer written before every step (each step timed alone)"
+        if self.rot == 1:
+            return "K cache of one step larger than 2x L2 (no rotation needed)"
+        return f"{self.rot} rotating buffer sets (K cache, W_KV, q, k) > 2x L2"
+
+    def footprint(self):
+        return {"k_only_bytes": int(self.B * self.cap * self.d * self.esz),
+                "k_plus_v_bytes": int(2 * self.B * self.cap * self.d * self.esz)}
 
 
-def run_sweep():
-    """Ordering (a) vs (b) over attended lengths T = 1K..128K (d=4096, H=32, B=1, no append), with
-    the K cache filled by the prompt-phase kernel, plus the 8192-token prompt projection. Each T is
-    timed with CUDA events behind a spin kernel (so the GPU never waits for the host), the result is
-    recorded in the SLIM_AUTO table and the ordering SLIM_AUTO then picks is reported."""
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def roofline_record(name, r):
+    return {"bound": "hbm", "achieved": r["achieved"], "peak": r["hbm_peak"], "unit": "GB/s",
+            "frac": (r["achieved"] / r["hbm_peak"]) if r["achieved"] else None,
+            "traffic": profile_traffic(name),
+            "kernel": "split kernel (streams the K cache; decode_b_tc_kernel for bf16, decode_simt_kernel for fp32)",
+            "bytes_per_launch": r["kernel_bytes"], "avg_launch_ms": r["split_ms"],
+            "peak_source": r["peak_src"] + " (MEASURED_PEAKS.json hbm_gbs, burst copy)"}
+
+
+def sub_record(name, S, dev, cpu_budget):
+    """One other workload at its own step count: the same measurements as the headline."""
+    import torch
+    w = WORKLOADS[name]
+    wl = Workload(name, S, dev, max_steps=max(w["steps"], 64) + 8)
+    r = wl.measure(w["steps"], 3)
+    rate, threads, n, T = cpu_oracle_rate(w, budget_s=cpu_budget)
+    rec = {"workload": w["desc"], "steps": w["steps"], "warmup": 3, "ms_per_step": r["ms_step"],
+           "steps_per_s": 1e3 / r["ms_step"], "tokens_per_s": 1e3 / r["ms_step"] * w["B"],
+           "step_hbm_gbs": r["step_bytes"] / (r["ms_step"] * 1e-3) / 1e9,
+           "step_frac": r["step_bytes"] / (r["ms_step"] * 1e-3) / 1e9 / r["hbm_peak"],
+           "ordering": {1: "a", 2: "b"}.get(r["chosen"], "?"), "launches_per_step": r["launches"],
+           "roofline": roofline_record(name, r),
+           "e2e": {"value": 1e3 / r["e2e_ms"], "unit": "steps/s"} if r["e2e_ms"] else None,
+           "l2": wl.l2_note(), "footprint": wl.footprint(), "status": r["status"],
+           "cpu_baseline": {"value": rate, "unit": "steps/s", "cores": threads, "kind": "oracle",
+                            "sample": f"{n} single-sequence float64 oracle steps at T={T}, scaled to the batch"}}
+    del wl
+    torch.cuda.empty_cache()
+    return rec
+
+
+def run_sweep(S, dev):
+    """Ordering (a) vs (b) over attended lengths T = 1K..128K (d=4096, H=32, B=1, no append), K cache
+    filled by the prompt-phase kernel; and the 8192 x 4096 x 4096 prompt projection. Each T is timed
+    with CUDA events behind a spin kernel (the GPU never waits for the host); the result goes into
+    the SLIM_AUTO table and the ordering SLIM_AUTO then picks is reported."""
     import torch
 
-    from only_cache_exact_b200 import params, slim as S, synth
-    dev = torch.device("cuda", 0)
+    from only_cache_exact_b200 import params, synth
     d, H, B = 4096, 32, 1
     Ts = [1024, 2048, 4096, 8192, 16384, 32768, 65536, 131072 - 64]
     cap = 131072
@@ -431,22 +524,27 @@ def run_sweep():
     K = torch.zeros(B, cap, d, dtype=torch.bfloat16, device=dev)
     lens = torch.zeros(B, dtype=torch.int32, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    # the 8192-token prompt: K = X·W_K into the cache (timed), then the rest of the cache in chunks
     chunk = 8192
-    X = synth.to_storage(synth.make_tokens(chunk, d, 0, 0, "bf16"), "bf16").to(dev).view(1, chunk, d)
+    X = synth.make_tokens_device(chunk, d, 1000, 0, "bf16", device=dev).view(1, chunk, d)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    S.slim_prefill_k(X, W_K, K, lens, status)
-    lens.zero_()
+    for _ in range(2):
+        lens.zero_()
+        S.slim_prefill_k(X, W_K, K, lens, status)
     torch.cuda.synchronize()
-    e0.record()
-    S.slim_prefill_k(X, W_K, K, lens, status)
-    e1.record()
-    e1.synchronize()
-    ms_p = e0.elapsed_time(e1)
-    print(json.dumps({"sweep": "prompt projection", "rows": chunk, "d": d, "ms": round(ms_p, 4),
-                      "tflops": round(2.0 * chunk * d * d / ms_p / 1e9, 1)}))
+    reps = 5
+    tot = 0.0
+    for _ in range(reps):
+        lens.zero_()
+        torch.cuda._sleep(int(5e6))
+        e0.record()
+        S.slim_prefill_k(X, W_K, K, lens, status)
+        e1.record()
+        e1.synchronize()
+        tot += e0.elapsed_time(e1)
+    ms_p = tot / reps
+    prefill = {"rows": chunk, "d": d, "ms": ms_p, "tflops": 2.0 * chunk * d * d / ms_p / 1e9}
     for r0 in range(chunk, cap, chunk):
-        Xr = synth.to_storage(synth.make_tokens(chunk, d, 1000 + r0, 0, "bf16"), "bf16").to(dev).view(1, chunk, d)
+        Xr = synth.make_tokens_device(chunk, d, 1000 + r0 // chunk, 0, "bf16", device=dev).view(1, chunk, d)
         S.slim_prefill_k(Xr, W_K, K, lens, status)
     torch.cuda.synchronize()
     x_new = synth.make_tokens(1, d, 0, 0, "bf16", part=2)
@@ -454,6 +552,7 @@ def run_sweep():
     out = torch.empty(B, d, dtype=torch.float32, device=dev)
     ws = S.alloc_workspace(S.SLIM_BF16, B, d, H, cap, S.SLIM_AUTO, device=dev)
     S.slim_tune_clear()
+    rows = []
     for T in Ts:
         ms = {}
         for name, v in (("a", S.SLIM_VARIANT_A), ("b", S.SLIM_VARIANT_B)):
@@ -471,46 +570,78 @@ def run_sweep():
             ms[name] = e0.elapsed_time(e1) / n
         S.slim_tune_record(S.SLIM_BF16, B, d, H, T, ms["a"], ms["b"])
         pick = S.slim_select_variant(S.SLIM_BF16, B, d, H, T)
-        kbytes = T * d * 2
-        print(json.dumps({"sweep": "ordering crossover", "d": d, "H": H, "B": B, "T": T,
-                          "ms_a": round(ms["a"], 5), "ms_b": round(ms["b"], 5),
-                          "b_hbm_gbs": round(kbytes / (ms["b"] * 1e-3) / 1e9, 1),
-                          "auto_picks": {1: "a", 2: "b"}[pick], "status": int(status.item())}))
+        step_bytes = T * d * 2 + d * d * 2 + 2 * d * 4
+        rows.append({"T": T, "ms_a": ms["a"], "ms_b": ms["b"], "a_over_b": ms["a"] / ms["b"],
+                     "b_step_hbm_gbs": step_bytes / (ms["b"] * 1e-3) / 1e9,
+                     "a_tflops": 2.0 * T * d * d / (ms["a"] * 1e-3) / 1e12,
+                     "auto_picks": {1: "a", 2: "b"}[pick]})
     S.slim_tune_clear()
+    st = int(status.item())
+    del K, ws
+    torch.cuda.empty_cache()
+    return {"d": d, "H": H, "B": B, "points": rows, "status": st}, prefill
 
 
-def cpu_oracle_rate(w, budget_s=12.0):
-    """Oracle step time on the host: float64 standard MHA with explicit K and V caches, one sequence
-    at a time (sequences are independent), as many steps as fit in the budget."""
-    from threadpoolctl import threadpool_info
+def run_prefill_d1024(S, dev):
+    """Prompt-phase projection of 8 sequences x 4096 rows at d=1024 (K = X·W_K)."""
+    import torch
 
-    from oracle import slim_oracle as O
     from only_cache_exact_b200 import synth
-    d, H = w["d"], w["H"]
-    lens = seq_lengths(w)
-    T = int(lens[0]) + (1 if w["append"] else 0)
-    rng = np.random.default_rng(0)
-    K = rng.standard_normal((T, d))
-    V = rng.standard_normal((T, d))
-    q = rng.standard_normal(d)
-    O.mha_decode(q, K, V, H)  # warm
-    n, t0 = 0, time.perf_counter()
-    while time.perf_counter() - t0 < budget_s:
-        O.mha_decode(q, K, V, H)
-        n += 1
-    per_seq = (time.perf_counter() - t0) / n
-    # one step = every sequence of the batch (ragged: scale by mean length)
-    step_s = per_seq * float(np.sum(lens + (1 if w["append"] else 0))) / T
-    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    return 1.0 / step_s, threads, n, T
+    B, n_rows, d = 8, 4096, 1024
+    X = synth.make_tokens_device(B * n_rows, d, 7, 0, "bf16", device=dev).view(B, n_rows, d)
+    W_K = synth.to_storage(synth.make_weights(d, 0, "bf16").W_K, "bf16").to(dev)
+    Kp = torch.empty(B, n_rows + 8, d, dtype=torch.bfloat16, device=dev)
+    lens = torch.zeros(B, dtype=torch.int32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    for _ in range(2):
+        lens.zero_()
+        S.slim_prefill_k(X, W_K, Kp, lens, status)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    tot, reps = 0.0, 5
+    for _ in range(reps):
+        lens.zero_()
+        torch.cuda._sleep(int(5e6))
+        e0.record()
+        S.slim_prefill_k(X, W_K, Kp, lens, status)
+        e1.record()
+        e1.synchronize()
+        tot += e0.elapsed_time(e1)
+    ms = tot / reps
+    return {"rows": B * n_rows, "d": d, "ms": ms, "tflops": 2.0 * B * n_rows * d * d / ms / 1e9}
 
 
+def run_variant_a(S, dev):
+    """Ordering (a) on the d=1024, B=8, T=4096 workload (materialise V = K·W_KV, then softmax·V)."""
+    import torch
+    wl = Workload("d1024_h16_b8_t4096", S, dev, max_steps=64)
+    n = 20
+    for i in range(3):
+        wl.step(i, S.SLIM_VARIANT_A)
+    wl.stream.synchronize()
+    wl.reset_lengths()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(wl.stream):
+        torch.cuda._sleep(int(20e6))
+        e0.record(wl.stream)
+        for i in range(n):
+            wl.step(i, S.SLIM_VARIANT_A)
+        e1.record(wl.stream)
+    e1.synchronize()
+    ms_a = e0.elapsed_time(e1) / n
+    rows = wl.rows_attended(n) / n
+    flops = 2.0 * rows * wl.d * wl.d
+    _, tc_peak, _ = peaks()
+    del wl
+    torch.cuda.empty_cache()
+    return {"ms_per_step": ms_a, "steps_per_s": 1e3 / ms_a, "tflops": flops / (ms_a * 1e-3) / 1e12,
+            "frac_of_bf16_peak": flops / (ms_a * 1e-3) / 1e12 / tc_peak}
+
+
+# ------------------------------------------------------------------------------------------ main
 def main():
     args = parse()
     w = WORKLOADS[args.workload]
-    if args.sweep:
-        run_sweep()
-        return
     if args.impl == "reference":
         # the oracle runs on rank 0's host cores only; no process group, no GPU
         if int(os.environ.get("RANK", "0")) != 0:
@@ -534,47 +665,61 @@ def main():
         print(json.dumps(line))
         return
 
-    r = run_ours(args, rank, world, local, pg)
+    import torch
+
+    from only_cache_exact_b200 import replicas, slim as S
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl = Workload(args.workload, S, dev, rank, world, max_steps=max(args.steps, args.warmup, 64) + 8,
+                  rot=args.rot)
+    sampler = ClockSampler(local)
+    r = wl.measure(args.steps, args.warmup, pg, sampler)
+    cfg = dict(workload_cfg)
+    cfg["l2"] = wl.l2_note()
+    cfg["attended_T_range"] = [int(np.min(wl.lens0)) + (1 if wl.append else 0),
+                               int(np.max(wl.lens0)) + (-(-args.steps // wl.rot) if wl.append else 0)]
+    h2d = int(w["B"] * w["d"] * 4 + (w["B"] * w["d"] * wl.esz if wl.append else 0))
+    d2h = int(w["B"] * w["d"] * 4)
+    footprint = wl.footprint()
+    del wl
+    torch.cuda.empty_cache()
+
+    extras = {}
+    if not args.no_extras and world == 1:
+        extras["workloads"] = {n: sub_record(n, S, dev, 3.0) for n in SUBRECORDS if n != args.workload}
+        extras["sweep"], extras["prefill"] = run_sweep(S, dev)
+        extras["prefill_d1024"] = run_prefill_d1024(S, dev)
+        extras["variant_a"] = run_variant_a(S, dev)
+
     if rank != 0:
         if pg:
             pg.destroy_process_group()
         return
-    from only_cache_exact_b200 import replicas
     steps_per_s = replicas.whole_job_rate(1, world, r["ms_step"])
-    tokens_per_s = steps_per_s * w["B"]
     cpu = None
     if world == 1 and not args.no_extras:
         rate, threads, n, T = cpu_oracle_rate(w)
         cpu = {"value": rate, "unit": "steps/s", "cores": threads, "kind": "oracle",
                "sample": f"{n} single-sequence float64 oracle steps at T={T} (explicit K and V), "
                          f"scaled to the B={w['B']} batch"}
-    trf = profile_traffic(f"decode_b_tc_{args.workload}.md")
-    roof = {"bound": "hbm", "achieved": r["achieved"], "peak": r["hbm_peak"], "unit": "GB/s",
-            "frac": (r["achieved"] / r["hbm_peak"]) if r["achieved"] else None,
-            "traffic": trf, "kernel": "decode_b_tc_kernel (split-T, streams the K cache)",
-            "bytes_per_launch": r["kernel_bytes"], "avg_launch_ms": r["split_avg_ms"],
-            "peak_source": r["peak_src"] + " (MEASURED_PEAKS.json hbm_gbs, burst copy)"}
-    cfg = dict(workload_cfg)
-    cfg["l2"] = f"{r['rot']} rotating buffer sets (K cache, W_KV, q, k) > 2x L2"
-    cfg["attended_T_range"] = r["t_range"]
     line = {"metric": METRIC, "value": steps_per_s, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": r["ms_step"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if w["dtype"] == "bf16" else "f32", "data": "synthetic",
             "config": cfg,
-            "tokens_per_s": tokens_per_s,
+            "tokens_per_s": steps_per_s * w["B"],
             "step_hbm_gbs": r["step_bytes"] / (r["ms_step"] * 1e-3) / 1e9,
+            "step_frac": r["step_bytes"] / (r["ms_step"] * 1e-3) / 1e9 / r["hbm_peak"],
             "ordering": {1: "a", 2: "b"}.get(r["chosen"], "?"),
-            "roofline": roof,
+            "roofline": roofline_record(args.workload, r),
             "cpu_baseline": cpu,
-            "e2e": {"value": replicas.whole_job_rate(1, world, r["e2e_ms"]), "unit": "steps/s", "h2d_bytes_per_step": r["h2d"],
-                    "d2h_bytes_per_step": r["d2h"]},
+            "e2e": {"value": replicas.whole_job_rate(1, world, r["e2e_ms"]), "unit": "steps/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": r["launches"] * args.steps,
             "launches_per_step": r["launches"],
-            "clocks": r["clocks"],
-            "footprint": {"k_only_bytes": int(w["B"] * r["cap"] * w["d"] * r["esz"]),
-                          "k_plus_v_bytes": int(2 * w["B"] * r["cap"] * w["d"] * r["esz"])},
-            "status": r["st"]}
-    line.update(r["extras"])
+            "clocks": sampler.summary(),
+            "footprint": footprint,
+            "status": r["status"]}
+    line.update(extras)
     print(json.dumps(line))
     if pg:
         pg.destroy_process_group()

@@ -137,22 +137,27 @@ int slim_decode_step_host(const float* q_host, const void* k_new_host, void* Kca
                           float* out_host, void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream);
 
 /*
- * slim_decode_step_noalloc — slim_decode_step without a caller workspace,
- * for callers that cannot allocate device memory (code that must not call
- * cudaMalloc, e.g. while a framework captures a CUDA graph or runs under a
- * fixed memory plan). The paper has no counterpart: this is a packaging of
- * the same step. Arguments and results are those of slim_decode_step minus
- * `workspace`/`ws_bytes`; this call itself allocates nothing.
+ * slim_decode_step_noalloc — slim_decode_step without a caller workspace, for
+ * callers that cannot allocate device memory: a plug-in whose host runtime
+ * owns all device memory under a plan fixed at start-up and passes it only
+ * the tensors it computes on, or a latency-critical decode loop that cannot
+ * afford cudaMalloc's implicit device synchronisation. The paper has no
+ * counterpart: it is a packaging of the same step. Arguments and results are
+ * those of slim_decode_step minus `workspace`/`ws_bytes`; the caller still
+ * passes every input and output. This call allocates nothing (no cudaMalloc,
+ * no cudaFree, no allocating library routine).
  *
  * Scratch: a buffer of SLIM_NOALLOC_SCRATCH_BYTES compiled into the library,
- * present on every GPU that loads it until the process exits. Sizes whose
- * slim_decode_workspace_bytes(...) exceeds it are rejected with
- * SLIM_EWORKSPACE before anything is launched. The first call on a device
- * looks up the buffer's device address (cudaGetSymbolAddress); make that
- * first call outside any stream capture. Every call on a device shares the
- * one buffer, which keeps the previous call's contents (the step needs no
- * zeroed scratch), so calls that overlap on the GPU, e.g. on two streams,
- * race with each other and must be serialised by the caller.
+ * held on every GPU that loads the library until the process exits. Sizes
+ * whose slim_decode_workspace_bytes(...) exceeds it are rejected with
+ * SLIM_EWORKSPACE before anything is enqueued. The first call on a device
+ * looks up the buffer's device address (cudaGetSymbolAddress, with that
+ * device current) and remembers it; make that first call before any stream
+ * capture. Every call on a device shares the one buffer, which keeps the
+ * previous call's contents: the step reads no scratch value it has not
+ * written in the same call, so nothing needs clearing, but calls that overlap
+ * on the GPU (e.g. on two streams) race with each other and must be
+ * serialised by the caller.
  */
 #define SLIM_NOALLOC_SCRATCH_BYTES (32 * 1024 * 1024)
 int slim_decode_step_noalloc(const float* q, const void* k_new, void* Kcache, int32_t* lens, const void* W_KV,

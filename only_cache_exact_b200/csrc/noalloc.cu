@@ -1,19 +1,21 @@
 // slim_decode_step_noalloc: the generation step for callers that cannot
-// allocate device memory, for example code running where cudaMalloc is
-// forbidden (inside CUDA-graph capture of a framework that owns all
-// allocations, or a runtime with a fixed memory plan). Its scratch is a
-// fixed buffer compiled into this library instead of a caller workspace.
+// allocate device memory. Some hosts hand a plug-in only the buffers it
+// computes on: an inference runtime that owns every byte of device memory
+// under a plan fixed at start-up, or a latency-critical decode loop in which
+// cudaMalloc's implicit device synchronisation is not acceptable. Such a
+// caller cannot provide the workspace slim_decode_step needs, so this entry
+// point takes its scratch from a fixed buffer compiled into this library.
 #include <cuda_runtime.h>
 
 #include <mutex>
 
 #include "slim_internal.h"
 
-namespace {
-
 // Scratch of the allocation-free entry point: SLIM_NOALLOC_SCRATCH_BYTES bytes
 // on every GPU that loads this library, held until the process exits.
-__device__ __align__(256) unsigned char g_noalloc_scratch[SLIM_NOALLOC_SCRATCH_BYTES];
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SLIM_NOALLOC_SCRATCH_BYTES];
+
+namespace {
 
 constexpr int kMaxDevices = 64;
 void* g_scratch_addr[kMaxDevices] = {};

@@ -214,6 +214,9 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
     flush();
   }
   const bool ok = __syncthreads_and(mbar_wait(wbar, 0u, p.status));
+  // after a wait that gave up, the block copy may still be landing in this CTA's shared memory:
+  // one more bounded wait keeps the CTA alive until it has (copies always complete)
+  if (!ok && tid == 0) mbar_wait(wbar, 0u, p.status);
 
   // ---- this CTA's product o_r[b, :] = ū[b, block] · W_KV[block, h-cols]
   if (ok && p.use_mma && nb > 4) {
@@ -449,7 +452,10 @@ __global__ void __launch_bounds__(kLeanThreads, 1)
   uint32_t ph = 0;
   for (int r0 = 0; r0 < n; r0 += p.cap_items, ph ^= 1u) {
     ok = __syncthreads_and(mbar_wait(ubar, ph, p.status));
-    if (!ok) break;
+    if (!ok) {
+      if (tid == 0) mbar_wait(ubar, ph, p.status);  // drain the staged copies before leaving
+      break;
+    }
     const int nr = min(n - r0, p.cap_items);
     for (int c = 0; c < nr; ++c) {
       const float w = ws_[r0 + c];
@@ -465,7 +471,9 @@ __global__ void __launch_bounds__(kLeanThreads, 1)
       if (warp == 0) lean_stage(us, p.U, lo, r0 + p.cap_items, n, p.cap_items, p.H, h, d, ubar, lane);
     }
   }
-  ok = __syncthreads_and(ok && mbar_wait(wbar, 0u, p.status));
+  const bool w_ok = __syncthreads_and(mbar_wait(wbar, 0u, p.status));
+  if (!w_ok && tid == 0) mbar_wait(wbar, 0u, p.status);  // the W_KV copy must land before exit
+  ok = ok && w_ok;
 
   // o[j] = Σ_rows ū[row] W[row][j]: this thread's rows, all 64 outputs
   float acc[kLeanDh];

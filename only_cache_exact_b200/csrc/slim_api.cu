@@ -378,8 +378,12 @@ int slim_decode_step(const float* q, const void* k_new, void* Kcache, int32_t* l
 int slim_decode_step_host(const float* q_host, const void* k_new_host, void* Kcache, int32_t* lens,
                           const void* W_KV, int dtype, int B, int d, int H, int64_t cap, int variant, int64_t t_hint,
                           float* out_host, void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream) {
-  if (!q_host || !out_host) return SLIM_EINVAL;
-  if (!valid_dims(dtype, B, d, H, cap)) return SLIM_EINVAL;
+  // every check slim_decode_step makes on its own arguments comes first, so that a rejected call
+  // has enqueued no copy
+  if (!q_host || !out_host || !Kcache || !lens || !W_KV || !dev_status) return SLIM_EINVAL;
+  if (!valid_dims(dtype, B, d, H, cap) || variant < SLIM_AUTO || variant > SLIM_VARIANT_B) return SLIM_EINVAL;
+  if (!aligned(Kcache, 16) || !aligned(W_KV, 16)) return SLIM_EINVAL;
+  if ((static_cast<size_t>(d) * esize(dtype)) % 16 != 0) return SLIM_EUNSUPPORTED;
   if (!workspace || !aligned(workspace, kAlign)) return SLIM_EWORKSPACE;
   const WsLayout wl = ws_layout(dtype, B, d, H, cap, variant);
   if (ws_bytes < wl.total) return SLIM_EWORKSPACE;

@@ -36,6 +36,7 @@ __all__ = [
     "LayerWeights",
     "make_weights",
     "make_tokens",
+    "make_tokens_device",
     "make_lengths",
 ]
 
@@ -107,6 +108,20 @@ def make_tokens(n: int, d: int, seed: int, seq: int, dtype: str = "bf16", part: 
     """
     rng = stream(seed, part, seq)
     return round_to(rng.standard_normal((n, d)), dtype)
+
+
+def make_tokens_device(n: int, d: int, seed: int, seq: int, dtype: str = "bf16", part: int = 1,
+                       device="cuda") -> torch.Tensor:
+    """n token rows X ~ N(0,1) of sequence `seq` drawn by torch's generator on `device`, in `dtype`.
+
+    For workloads whose prompts are too large to draw on the host (tens of
+    millions of rows). The stream is seeded from (seed, part, seq) like
+    `make_tokens` but is a different stream: a test that needs these rows on
+    the host copies them back (they are exact in `dtype`)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(int(np.random.SeedSequence([int(seed), int(part), int(seq)]).generate_state(1, np.uint64)[0]
+                      & 0x7FFFFFFFFFFFFFFF))
+    return torch.randn(n, d, generator=g, device=device, dtype=torch.float32).to(_TORCH_DTYPES[dtype])
 
 
 def make_lengths(batch: int, lo: int, hi: int, seed: int) -> np.ndarray:

@@ -44,7 +44,6 @@ __all__ = [
     "softmax",
     "head_slice",
     "mha_decode",
-    "mha_decode_batch",
     "wkv_closed_form",
     "wkv_solve",
     "slim_decode_a",
@@ -90,11 +89,6 @@ def mha_decode(q: np.ndarray, K: np.ndarray, V: np.ndarray, H: int) -> np.ndarra
         p = softmax(K[:, c] @ q[c] / np.sqrt(d_h))
         o[c] = p @ V[:, c]
     return o
-
-
-def mha_decode_batch(q: np.ndarray, Ks, Vs, H: int) -> np.ndarray:
-    """`mha_decode` for each sequence b of a batch; Ks/Vs are per-sequence (T_b, d) arrays."""
-    return np.stack([mha_decode(q[b], Ks[b], Vs[b], H) for b in range(len(Ks))])
 
 
 def wkv_closed_form(G_orth: np.ndarray, s: np.ndarray, W_V: np.ndarray) -> np.ndarray:

@@ -7,6 +7,7 @@ only_cache_exact_b200.synth; expected values only from oracle/.
 """
 from __future__ import annotations
 
+import functools
 from dataclasses import dataclass, field
 
 import numpy as np
@@ -38,9 +39,15 @@ class Case:
         return len(self.lens)
 
 
+@functools.lru_cache(maxsize=8)
+def weights(d, seed, dtype) -> synth.LayerWeights:
+    """synth.make_weights, memoised (a d=4096 layer takes seconds to draw)."""
+    return synth.make_weights(d, seed, dtype)
+
+
 def make_case(d, H, lens, cap, dtype="bf16", append=True, seed=0) -> Case:
     c = Case(d=d, H=H, lens=np.asarray(lens, dtype=np.int32), cap=cap, dtype=dtype, append=append, seed=seed)
-    c.w = synth.make_weights(d, seed, dtype)
+    c.w = weights(d, seed, dtype)
     c.X = [synth.make_tokens(int(n), d, seed, b, dtype) for b, n in enumerate(c.lens)]
     c.x_new = np.stack([synth.make_tokens(1, d, seed, b, dtype, part=2)[0] for b in range(c.B)])
     c.q64 = c.x_new @ c.w.W_Q
@@ -118,3 +125,48 @@ def rel_l2_per_head(got: np.ndarray, ref: np.ndarray, H: int) -> np.ndarray:
     g = got.reshape(B, H, d // H)
     r = ref.reshape(B, H, d // H)
     return np.linalg.norm(g - r, axis=2) / np.maximum(np.linalg.norm(r, axis=2), 1e-30)
+
+
+class BigState:
+    """A full-size workload: prompt rows drawn on the device (synth.make_tokens_device), the K
+    cache filled by slim_prefill_k in chunks, and host copies of the rows of the sequences in
+    `sample` only, so the oracle can recompute those sequences one at a time. The Case it
+    carries holds X for the sampled sequences alone (oracle_out(c, sample) works on it)."""
+
+    def __init__(self, d, H, lens, cap, S, sample, append=True, seed=0, chunk=8192, dev="cuda"):
+        c = Case(d=d, H=H, lens=np.asarray(lens, dtype=np.int32), cap=cap, dtype="bf16", append=append, seed=seed)
+        c.w = weights(d, seed, "bf16")
+        self.S, self.c, self.sample = S, c, list(sample)
+        self.K = torch.empty(c.B, cap, d, dtype=torch.bfloat16, device=dev)
+        self.lens = torch.zeros(c.B, dtype=torch.int32, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        W_K = synth.to_storage(c.w.W_K, "bf16").to(dev)
+        c.X = [None] * c.B
+        for b in range(c.B):
+            n = int(c.lens[b])
+            rows = []
+            for r0 in range(0, n, chunk):
+                r1 = min(n, r0 + chunk)
+                Xd = synth.make_tokens_device(r1 - r0, d, seed + 1000 * (1 + r0 // chunk), b, "bf16", device=dev)
+                S.slim_prefill_k(Xd.view(1, r1 - r0, d), W_K, self.K[b:b + 1], self.lens[b:b + 1], self.status)
+                if b in self.sample:
+                    rows.append(Xd.float().cpu().double().numpy())
+            if b in self.sample:
+                c.X[b] = np.vstack(rows) if rows else np.zeros((0, d))
+        c.x_new = np.stack([synth.make_tokens(1, d, seed, b, "bf16", part=2)[0] for b in range(c.B)])
+        c.q64 = c.x_new @ c.w.W_Q
+        c.k_new64 = c.x_new @ c.w.W_K
+        self.W_KV = params.make_wkv(c.w.W_K, c.w.W_V, dtype=torch.bfloat16, device=dev)
+        self.q = torch.from_numpy(c.q64).to(torch.float32).to(dev).contiguous()
+        self.k_new = synth.to_storage(synth.round_to(c.k_new64, "bf16"), "bf16").to(dev) if append else None
+        self.out = torch.full((c.B, d), float("nan"), dtype=torch.float32, device=dev)
+        self.ws = S.alloc_workspace(S.SLIM_BF16, c.B, d, H, cap, S.SLIM_VARIANT_B, device=dev)
+        torch.cuda.synchronize()
+        assert int(self.status.item()) == 0
+        assert torch.equal(self.lens.cpu(), torch.from_numpy(c.lens))
+
+    def step(self, variant):
+        self.S.slim_decode_step(self.q, self.k_new, self.K, self.lens, self.W_KV, self.c.H, self.out, self.ws,
+                                self.status, variant=variant)
+        torch.cuda.synchronize()
+        return self.out.cpu().double().numpy()

@@ -94,11 +94,39 @@ def test_prefill_rejects_bad_arguments(S):
     assert L.slim_prefill_k(f, f, f, f, 3, 1, 8, 256, 64, f, None) == S.SLIM_EINVAL
 
 
-def test_host_entry_rejects_null_host_buffers(S):
+def test_host_entry_rejects_bad_arguments_before_any_copy(S):
+    """Every argument check precedes the host-to-device copies: with fake device pointers that
+    would fault if a copy were enqueued, a bad call returns its error code and does nothing."""
     L = S.raw_lib()
     f = ctypes.c_void_p(1 << 20)
-    assert L.slim_decode_step_host(None, None, f, f, f, S.SLIM_BF16, 8, 1024, 16, 4160, 0, 0, f, f, 1 << 40, f,
-                                   None) == S.SLIM_EINVAL
+    h = ctypes.c_void_p(2 << 20)
+
+    def call(q=h, K=f, lens=f, w=f, v=0, d=1024, st=f):
+        return L.slim_decode_step_host(q, None, K, lens, w, S.SLIM_BF16, 8, d, 16, 4160, v, 0, h, f, 1 << 40,
+                                       st, None)
+
+    assert call(q=None) == S.SLIM_EINVAL
+    assert call(K=None) == S.SLIM_EINVAL
+    assert call(lens=None) == S.SLIM_EINVAL
+    assert call(w=None) == S.SLIM_EINVAL
+    assert call(st=None) == S.SLIM_EINVAL
+    assert call(v=7) == S.SLIM_EINVAL
+    assert call(v=-1) == S.SLIM_EINVAL
+    assert call(d=1000) == S.SLIM_EINVAL
+    assert call(K=ctypes.c_void_p((1 << 20) + 8)) == S.SLIM_EINVAL  # cache not 16-byte aligned
+
+
+def test_binding_constants_match_the_header(S):
+    """The Python constants restate include/slim.h's #defines; a changed header must not drift."""
+    src = open(os.path.join(ROOT, "include", "slim.h")).read()
+    defs = {}
+    for name, val in re.findall(r"#define[ \t]+(SLIM_[A-Z_0-9]+)[ \t]+(.+)", src):
+        val = re.sub(r"/\*.*?\*/", "", val).strip()
+        defs[name] = eval(val, {})  # integer literals and products only
+    assert defs, "no #define found"
+    for name, val in defs.items():
+        assert hasattr(S, name), name
+        assert getattr(S, name) == val, (name, getattr(S, name), val)
 
 
 def test_ordering_table(S):
