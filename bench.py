@@ -77,6 +77,7 @@ WORKLOADS = {
 DEFAULT = "d4096_h32_b16_t16k_32k"
 SUBRECORDS = ["d256_h4_b1_t128_f32", "d1024_h16_b8_t4096", "d1280_h20_b64_t1500_cross", "d4096_h32_b1_t8192",
               "d4096_h32_b1_t131072"]
+KV_BASELINE = ["d1024_h16_b8_t4096", "d4096_h32_b16_t16k_32k", "d1280_h20_b64_t1500_cross", "d4096_h32_b1_t131072"]
 FLUSH_BYTES = 256 << 20
 
 
@@ -88,6 +89,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT, choices=sorted(WORKLOADS))
     ap.add_argument("--rot", type=int, default=0, help="buffer sets rotated (0: automatic)")
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling runs)")
     ap.add_argument("--no-extras", action="store_true", help="headline line only (no sub-records, sweep, CPU legs)")
     ap.add_argument("--ref-seconds", type=float, default=20.0, help="CPU time budget of --impl reference")
     return ap.parse_args()
@@ -233,12 +235,15 @@ def cpu_oracle_rate(w, budget_s=12.0):
 class Workload:
     """Device state of one workload: K cache(s) filled by the prompt-phase kernel, W_KV, step inputs."""
 
-    def __init__(self, name, S, dev, rank=0, world=1, max_steps=256, rot=0):
+    def __init__(self, name, S, dev, rank=0, world=1, max_steps=256, rot=0, mha=False, batch=0):
         import torch
 
         from only_cache_exact_b200 import params, replicas, synth
         self.name, self.S, self.dev = name, S, dev
-        w = self.w = WORKLOADS[name]
+        w = self.w = dict(WORKLOADS[name])
+        if batch:
+            w["B"] = batch
+        self.mha = mha  # standard MHA step over K and V caches (the baseline) instead of the Slim step
         d, H, B = w["d"], w["H"], w["B"]
         self.d, self.H, self.B = d, H, B
         self.append = w["append"]
@@ -247,7 +252,7 @@ class Workload:
         self.tdt = torch.bfloat16 if w["dtype"] == "bf16" else torch.float32
         self.dt_code = S.SLIM_BF16 if w["dtype"] == "bf16" else S.SLIM_F32
         self.esz = 2 if w["dtype"] == "bf16" else 4
-        set_bytes = int(np.sum(self.lens0)) * d * self.esz + d * d * self.esz
+        set_bytes = int(np.sum(self.lens0)) * d * self.esz * (2 if mha else 1) + (0 if mha else d * d * self.esz)
         l2 = torch.cuda.get_device_properties(dev).L2_cache_size
         if rot:
             self.rot = rot
@@ -269,7 +274,10 @@ class Workload:
         W_KV0 = params.make_wkv(wts.W_K, wts.W_V, dtype=self.tdt, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         K0 = torch.zeros(B, self.cap, d, dtype=self.tdt, device=dev)
+        V0 = torch.zeros(B, self.cap, d, dtype=self.tdt, device=dev) if mha else None
+        W_V = synth.to_storage(synth.round_to(wts.W_V, w["dtype"]), w["dtype"]).to(dev) if mha else None
         lens_dev0 = torch.zeros(B, dtype=torch.int32, device=dev)
+        lens_v = torch.zeros(B, dtype=torch.int32, device=dev)
         t = time.perf_counter()
         for b in range(B):
             n = int(self.lens0[b])
@@ -277,6 +285,8 @@ class Workload:
                 r1 = min(n, r0 + 8192)
                 Xb = synth.make_tokens_device(r1 - r0, d, 1000 + r0 // 8192, gids[b], w["dtype"], device=dev)
                 S.slim_prefill_k(Xb.view(1, r1 - r0, d), self.W_K, K0[b:b + 1], lens_dev0[b:b + 1], self.status)
+                if mha:
+                    S.slim_prefill_k(Xb.view(1, r1 - r0, d), W_V, V0[b:b + 1], lens_v[b:b + 1], self.status)
         torch.cuda.synchronize()
         self.fill_s = time.perf_counter() - t
         self.lens_dev0 = lens_dev0
@@ -284,13 +294,20 @@ class Workload:
         self.q0 = torch.from_numpy(x_new @ wts.W_Q).float().to(dev)
         self.k0 = (synth.to_storage(synth.round_to(x_new @ wts.W_K, w["dtype"]), w["dtype"]).to(dev)
                    if self.append else None)
+        self.v0 = (synth.to_storage(synth.round_to(x_new @ wts.W_V, w["dtype"]), w["dtype"]).to(dev)
+                   if self.append and mha else None)
         self.sets = []
         for i in range(self.rot):
-            self.sets.append(dict(K=K0 if i == 0 else K0.clone(), lens=lens_dev0.clone(),
-                                  W_KV=W_KV0 if i == 0 else W_KV0.clone(),
-                                  q=self.q0.clone(), k=None if self.k0 is None else self.k0.clone(),
-                                  out=torch.empty(B, d, dtype=torch.float32, device=dev),
-                                  ws=S.alloc_workspace(self.dt_code, B, d, H, self.cap, S.SLIM_AUTO, device=dev)))
+            st_ = dict(K=K0 if i == 0 else K0.clone(), lens=lens_dev0.clone(),
+                       q=self.q0.clone(), k=None if self.k0 is None else self.k0.clone(),
+                       out=torch.empty(B, d, dtype=torch.float32, device=dev))
+            if mha:
+                st_.update(V=V0 if i == 0 else V0.clone(), v=None if self.v0 is None else self.v0.clone(),
+                           ws=S.alloc_mha_workspace(self.dt_code, B, d, H, self.cap, device=dev))
+            else:
+                st_.update(W_KV=W_KV0 if i == 0 else W_KV0.clone(),
+                           ws=S.alloc_workspace(self.dt_code, B, d, H, self.cap, S.SLIM_AUTO, device=dev))
+            self.sets.append(st_)
         self.t_hint = int(np.max(self.lens0))
         self.stream = torch.cuda.Stream(device=dev)
         self.flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev) if self.flush else None
@@ -299,6 +316,10 @@ class Workload:
     def step(self, i, variant=None):
         S = self.S
         s = self.sets[i % self.rot]
+        if self.mha:
+            S.slim_mha_decode_step(s["q"], s["k"], s["v"], s["K"], s["V"], s["lens"], self.H, s["out"], s["ws"],
+                                   self.status)
+            return
         S.slim_decode_step(s["q"], s["k"], s["K"], s["lens"], s["W_KV"], self.H, s["out"], s["ws"], self.status,
                            variant=S.SLIM_AUTO if variant is None else variant, t_hint=self.t_hint)
 
@@ -317,9 +338,10 @@ class Workload:
         """(split kernel bytes per launch, step bytes) averaged over nsteps steps: K rows attended
         (incl. the appended one) read once, q, k_new read and written; the step adds W_KV once and
         the output."""
-        per_step_const = self.B * self.d * 4 + (2 * self.B * self.d * self.esz if self.append else 0)
-        kernel = self.rows_attended(nsteps) * self.d * self.esz / nsteps + per_step_const
-        return kernel, kernel + self.d * self.d * self.esz + self.B * self.d * 4
+        caches = 2 if self.mha else 1
+        per_step_const = self.B * self.d * 4 + (2 * caches * self.B * self.d * self.esz if self.append else 0)
+        kernel = caches * self.rows_attended(nsteps) * self.d * self.esz / nsteps + per_step_const
+        return kernel, kernel + (0 if self.mha else self.d * self.d * self.esz) + self.B * self.d * 4
 
     def time_steps(self, K_steps, W_steps, pg=None, sample_clocks=None):
         """Device time of exactly K_steps steps after W_steps warm-up steps (ms)."""
@@ -445,7 +467,7 @@ class Workload:
         chosen = S.slim_select_variant(self.dt_code, self.B, self.d, self.H, self.t_hint)
         launches = S.slim_last_launch_count()
         n_live = min(max(K_steps, 8), 64)
-        split_ms = self.split_kernel_ms(n_live)
+        split_ms = None if self.mha else self.split_kernel_ms(n_live)
         kbytes, sbytes_live = self.algorithmic_bytes(n_live)
         _, sbytes = self.algorithmic_bytes(K_steps)
         hbm_peak, _, peak_src = peaks()
@@ -453,7 +475,7 @@ class Workload:
         r = dict(ms_step=ms_step, status=st, chosen=chosen, launches=launches, split_ms=split_ms,
                  kernel_bytes=int(kbytes), step_bytes=int(sbytes), achieved=achieved, hbm_peak=hbm_peak,
                  peak_src=peak_src)
-        r["e2e_ms"] = self.e2e_ms(max(8, min(K_steps, 200)), pg) if e2e else None
+        r["e2e_ms"] = self.e2e_ms(max(8, min(K_steps, 200)), pg) if e2e and not self.mha else None
         return r
 
     def l2_note(self):
@@ -502,6 +524,26 @@ def sub_record(name, S, dev, cpu_budget):
            "l2": wl.l2_note(), "footprint": wl.footprint(), "status": r["status"],
            "cpu_baseline": {"value": rate, "unit": "steps/s", "cores": threads, "kind": "oracle",
                             "sample": f"{n} single-sequence float64 oracle steps at T={T}, scaled to the batch"}}
+    del wl
+    torch.cuda.empty_cache()
+    return rec
+
+
+def kv_record(name, S, dev, slim_ms):
+    """The standard MHA step over explicit K and V caches (slim_mha_decode_step) on the same workload,
+    against the Slim step's ms per step: the pages' claim (up to 2x when memory-bound) as a ratio."""
+    import torch
+    w = WORKLOADS[name]
+    steps = min(w["steps"], 64)
+    wl = Workload(name, S, dev, max_steps=steps + 8, mha=True)
+    ms = wl.time_steps(steps, 3) / steps
+    _, sbytes = wl.algorithmic_bytes(steps)
+    hbm_peak, _, _ = peaks()
+    rec = {"workload": w["desc"], "steps": steps, "ms_per_step": ms, "steps_per_s": 1e3 / ms,
+           "step_hbm_gbs": sbytes / (ms * 1e-3) / 1e9, "step_frac": sbytes / (ms * 1e-3) / 1e9 / hbm_peak,
+           "kv_cache_bytes": int(2 * wl.B * wl.cap * wl.d * wl.esz), "l2": wl.l2_note(),
+           "slim_ms_per_step": slim_ms, "slim_speedup": ms / slim_ms if slim_ms else None,
+           "status": int(wl.status.item())}
     del wl
     torch.cuda.empty_cache()
     return rec
@@ -671,7 +713,11 @@ def main():
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     wl = Workload(args.workload, S, dev, rank, world, max_steps=max(args.steps, args.warmup, 64) + 8,
-                  rot=args.rot)
+                  rot=args.rot, batch=args.batch)
+    if args.batch:  # a reduced batch for profiling captures; the line says so
+        w = wl.w
+        workload_cfg["B"] = w["B"]
+        workload_cfg["workload"] += f" (batch reduced to {w['B']})"
     sampler = ClockSampler(local)
     r = wl.measure(args.steps, args.warmup, pg, sampler)
     cfg = dict(workload_cfg)
@@ -687,6 +733,10 @@ def main():
     extras = {}
     if not args.no_extras and world == 1:
         extras["workloads"] = {n: sub_record(n, S, dev, 3.0) for n in SUBRECORDS if n != args.workload}
+        slim_ms = {n: rec["ms_per_step"] for n, rec in extras["workloads"].items()}
+        slim_ms[args.workload] = r["ms_step"]
+        extras["kv_baseline"] = {n: kv_record(n, S, dev, slim_ms.get(n))
+                                 for n in KV_BASELINE if WORKLOADS[n]["dtype"] == "bf16"}
         extras["sweep"], extras["prefill"] = run_sweep(S, dev)
         extras["prefill_d1024"] = run_prefill_d1024(S, dev)
         extras["variant_a"] = run_variant_a(S, dev)

@@ -165,6 +165,32 @@ int slim_decode_step_noalloc(const float* q, const void* k_new, void* Kcache, in
                              int32_t* dev_status, void* stream);
 
 /*
+ * slim_mha_decode_step — the standard multi-head attention generation step
+ * over explicit K and V caches, the step Slim attention rewrites: for every
+ * sequence b and head h, o[b, h-cols] = softmax(q_h·K_h^T/sqrt(d_h))·V_h.
+ * Source: section "K-Cache is All You Need" (standard MHA caches k and v of
+ * every token; the article and the paper's abstract compare the K-only step
+ * with it: half the context memory, up to 2x faster when the step is
+ * memory-bandwidth-bound). Provided as the measured baseline of that claim.
+ *
+ *   q              float[B][d]          (device, read)
+ *   k_new, v_new   [B][d] bf16          this step's key and value, appended at
+ *                  row lens[b] of both caches before attending; both NULL =
+ *                  no append (attend over lens[b] rows, lens unchanged)
+ *   Kcache, Vcache [B][cap][d] bf16     (device; row lens[b] written when appending)
+ *   lens           int32[B]             (device; += 1 per appended sequence)
+ *   dtype          SLIM_BF16 only (SLIM_F32 returns SLIM_EUNSUPPORTED)
+ *   B, d, H        d % 256 == 0, d_h = d/H of 64 or 128
+ *   out            float[B][d]          (device, written); zero for a skipped sequence
+ *   workspace      >= slim_mha_decode_workspace_bytes(...), 256-byte aligned
+ *   dev_status     device int32 (SLIM_DEV_* bits, as for slim_decode_step)
+ */
+size_t slim_mha_decode_workspace_bytes(int dtype, int B, int d, int H, int64_t cap);
+int slim_mha_decode_step(const float* q, const void* k_new, const void* v_new, void* Kcache, void* Vcache,
+                         int32_t* lens, int dtype, int B, int d, int H, int64_t cap, float* out, void* workspace,
+                         size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/*
  * slim_tune — fills the SLIM_AUTO table for (dtype, B, d, H) by timing both
  * orderings, without append, at each attended length Ts[i] (1 <= Ts[i] <= cap)
  * with CUDA events on `stream`, `reps` repetitions each. It overwrites

@@ -2,15 +2,16 @@
 //
 // Slim Attention article, section "K-Cache is All You Need", generation
 // phase, second option: multiply the per-head softmax rows by K first (a full
-// d-row per head) and only then by W_KV. Per work item (one row chunk of one
-// sequence, see split_plan.cuh) this kernel streams the chunk's K rows once
-// and produces the flash-decoding partial of every head h:
+// d-row per head) and only then by W_KV. Per segment (the rows of one
+// sequence within a work group's contiguous share of all attended rows, see
+// split_plan.cuh) this kernel streams the segment's K rows once and produces
+// the flash-decoding partial of every head h:
 //     m_h = running max of the scaled scores (log2 domain)
 //     l_h = sum_t 2^(s_ht - m_h)
 //     U_h = sum_t 2^(s_ht - m_h) · K_t            (a full d-row, fp32)
 // reduce.cu merges the partials and applies W_KV.
 //
-// A cluster of CL CTAs shares one work item; CTA r owns the columns
+// A cluster of CL CTAs is one work group; CTA r owns the columns
 // [r·dS, (r+1)·dS), dS = d/CL <= 1024, and the heads whose columns lie there.
 // Per CTA (16 warps):
 //   warp 0       TMA producer: a K tile is TT rows x dS columns, one 3-D box
@@ -74,7 +75,6 @@ struct DecodeTCParams {
   int64_t cap;
   int append;
   int n_groups;   // clusters launched
-  int max_items;  // work items the workspace holds
   int stages;
   int min_rows;
   uint32_t tmem_cols;
@@ -102,8 +102,8 @@ __host__ __device__ inline TCSmem tc_smem_layout(int CL, int TT, int d, int stag
   o += (5u * stages + 2u) * 8u;
   s.slot_off = o;
   o += 16u;
-  s.plan_off = o;
-  o += 3u * static_cast<uint32_t>(B + 1) * 4u;
+  s.plan_off = o;  // s_nb [B + 1], s_q [B + 1], s_soff [B + 1], s_plan [2]
+  o += (3u * static_cast<uint32_t>(B + 1) + 2u) * 4u;
   s.total = o + 1024u;  // slack for aligning the base to 1024 bytes
   return s;
 }
@@ -180,12 +180,13 @@ __global__ void __launch_bounds__(kTCThreads, 1)
   uint64_t* pfull = bars + 2 * stages;         // P and alpha of every head of the cluster in place
   uint64_t* pempty = bars + 3 * stages;        // every CTA's MMAs done with the P stage, alphas read
   uint64_t* corr = bars + 4 * stages;          // accumulator corrected for this tile's new maxima
-  uint64_t* accfull = bars + 5 * stages;       // last MMA of an item completed
+  uint64_t* accfull = bars + 5 * stages;       // last MMA of a segment completed
   uint64_t* accempty = bars + 5 * stages + 1;  // epilogue finished reading the accumulator
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.slot_off);
   int* s_nb = reinterpret_cast<int*>(smem + L.plan_off);
-  int* s_rows = s_nb + (p.B + 1);
-  int* s_off = s_rows + (p.B + 1);
+  unsigned* s_q = reinterpret_cast<unsigned*>(s_nb + (p.B + 1));
+  unsigned* s_soff = s_q + (p.B + 1);
+  unsigned* s_plan = s_soff + (p.B + 1);
   const uint32_t kstage_bytes = static_cast<uint32_t>(TT) * dS * 2u;
   const uint32_t pstage_bytes = static_cast<uint32_t>(kPRows) * TT * 2u;
   // K stage layout: [TT/16 slabs][ncb column blocks][16 rows][128 bytes], 128-byte swizzled
@@ -225,24 +226,25 @@ __global__ void __launch_bounds__(kTCThreads, 1)
   pdl_wait_primary();
   pdl_launch_dependents();
   if (warp == 0)
-    plan_split(p.lens, p.B, p.cap, p.append, p.n_groups, p.max_items, p.min_rows, s_nb, s_rows, s_off, p.ws_meta,
-               p.status, blockIdx.x == 0);
+    plan_lean(p.lens, p.B, 1, p.cap, p.append, p.n_groups, p.min_rows, s_nb, s_q, s_soff, s_plan, p.ws_meta, p.status,
+              blockIdx.x == 0);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   if (CL > 1) cluster_sync();
   const uint32_t tmem = *tmem_slot;
-  const int n_items = s_off[p.B];
+  LeanCursor cur;  // this group's segments (every role walks the same list)
+  cur.init(group, p.B, s_q, s_plan);
+  SplitItem it;
   auto tiles_of = [&](const SplitItem& it) { return (it.row1 - it.row0 + TT - 1) / TT; };
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       const uint64_t pol = l2_policy_evict_first();
-      int g = 0;  // tiles issued so far (all items)
+      int g = 0;  // tiles issued so far (all segments)
       bool ok = true;
-      for (int item = group; item < n_items && ok; item += p.n_groups) {
-        const SplitItem it = plan_lookup(item, p.B, s_nb, s_rows, s_off);
+      while (ok && cur.next(it, s_nb, s_q, s_soff)) {
         const int nt = tiles_of(it);
         for (int t = 0; t < nt; ++t, ++g) {
           const int s = g % stages;
@@ -271,10 +273,9 @@ __global__ void __launch_bounds__(kTCThreads, 1)
       const uint32_t kbase = smem_u32(kst), pbase = smem_u32(pst);
       int g = 0, ii = 0;
       bool ok = true;
-      for (int item = group; item < n_items && ok; item += p.n_groups, ++ii) {
-        const SplitItem it = plan_lookup(item, p.B, s_nb, s_rows, s_off);
+      while (ok && cur.next(it, s_nb, s_q, s_soff)) {
         const int nt = tiles_of(it);
-        // the previous item's epilogue must have read the accumulator
+        // the previous segment's epilogue must have read the accumulator
         if (ii > 0 && !mbar_wait(accempty, static_cast<uint32_t>(ii - 1) & 1u, p.status)) break;
         for (int t = 0; t < nt; ++t, ++g) {
           const int s = g % stages;
@@ -326,10 +327,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
           else umma_commit(&pempty[s]);
         }
         umma_commit(accfull);  // also after a failed tile: covers every MMA issued so far
-        if (!ok) {
-          ++ii;
-          break;
-        }
+        ++ii;
       }
       // no MMA may be in flight at teardown: wait for the last commit
       if (ii > 0) mbar_wait(accfull, static_cast<uint32_t>(ii - 1) & 1u, p.status);
@@ -346,8 +344,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
     const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     int g = 0, ii = 0;
     bool ok = true;
-    for (int item = group; item < n_items && ok; item += p.n_groups, ++ii) {
-      const SplitItem it = plan_lookup(item, p.B, s_nb, s_rows, s_off);
+    for (; ok && cur.next(it, s_nb, s_q, s_soff); ++ii) {
       const int nt = tiles_of(it);
       for (int t = 0; t < nt; ++t, ++g) {
         const int s = g % stages;
@@ -381,10 +378,10 @@ __global__ void __launch_bounds__(kTCThreads, 1)
         if (lane == 0) mbar_arrive(&corr[s]);
       }
       if (!ok) break;
-      // epilogue: accumulator rows -> partial U[item][head][own columns]
+      // epilogue: accumulator rows -> partial U[slot][head][own columns]
       if (!__all_sync(0xffffffffu, mbar_wait(accfull, static_cast<uint32_t>(ii) & 1u, p.status))) break;
       tc_fence_after();
-      float* dst = p.ws_U + (static_cast<size_t>(item) * p.H + max(n, 0)) * p.d + col0 + 512 * hf;
+      float* dst = p.ws_U + (static_cast<size_t>(it.slot) * p.H + max(n, 0)) * p.d + col0 + 512 * hf;
       // four 16-column loads in flight per wait (hcols and my_cols are multiples of 64)
       for (int c = 0; c < hcols; c += 64) {
         float v[4][16];
@@ -425,8 +422,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
     }
     int g = 0;
     bool ok = true;
-    for (int item = group; item < n_items && ok; item += p.n_groups) {
-      const SplitItem it = plan_lookup(item, p.B, s_nb, s_rows, s_off);
+    while (ok && cur.next(it, s_nb, s_q, s_soff)) {
       const int nt = tiles_of(it);
       const int b = it.b;
       const int nb_old = it.nb - p.append;  // rows holding cached keys
@@ -676,7 +672,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
         }
       }
       if (!ok) break;
-      const size_t slot = static_cast<size_t>(item);
+      const size_t slot = static_cast<size_t>(it.slot);
 #pragma unroll
       for (int ps = 0; ps < NPASS; ++ps) {
         const int k = ps * HPP + hslot;
@@ -871,7 +867,6 @@ cudaError_t launch_decode_b_tc(const DecodeArgs& a, const SplitWorkspace& ws, cu
   prm.cap = a.cap;
   prm.append = a.k_new != nullptr ? 1 : 0;
   prm.n_groups = num_sms() / c.CL;
-  prm.max_items = ws.max_items;
   prm.stages = c.stages;
   prm.min_rows = max(16, 8 * a.H);
   prm.tmem_cols = c.tmem_cols;

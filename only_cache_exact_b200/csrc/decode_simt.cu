@@ -62,7 +62,7 @@ __host__ __device__ inline size_t simt_smem_bytes(int d, int H, int B, bool with
              + static_cast<size_t>(with_v ? d : H * d)   // accumulator
              + 2 * static_cast<size_t>(H) * kSimtRows    // scores, p
              + 3 * static_cast<size_t>(H);               // m, l, alpha
-  return f * 4 + ((tiles + 15) & ~size_t(15)) + 3 * static_cast<size_t>(B + 1) * 4 + 16;
+  return f * 4 + ((tiles + 15) & ~size_t(15)) + (3 * static_cast<size_t>(B + 1) + 2) * 4 + 16;
 }
 
 template <typename KT, bool VARIANT_A>
@@ -81,99 +81,104 @@ __global__ void __launch_bounds__(256) decode_simt_kernel(const SimtParams p) {
   float* alph = lsum + H;
   int* s_nb = reinterpret_cast<int*>(
       (reinterpret_cast<uintptr_t>(ks + kSimtRows * d * (VARIANT_A ? 2 : 1)) + 15) & ~uintptr_t(15));
-  int* s_rows = s_nb + (p.B + 1);
-  int* s_off = s_rows + (p.B + 1);
+  unsigned* s_q = reinterpret_cast<unsigned*>(s_nb + (p.B + 1));
+  unsigned* s_soff = s_q + (p.B + 1);
+  unsigned* s_plan = s_soff + (p.B + 1);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   if (warp == 0)
-    plan_split(p.lens, p.B, p.cap, p.attend_add, p.n_slots, p.n_slots, p.min_rows, s_nb, s_rows, s_off, p.ws_meta,
-               p.status, blockIdx.x == 0);
+    plan_lean(p.lens, p.B, 1, p.cap, p.attend_add, p.n_slots, p.min_rows, s_nb, s_q, s_soff, s_plan, p.ws_meta,
+              p.status, blockIdx.x == 0);
   __syncthreads();
-  const SplitItem it = plan_lookup(blockIdx.x, p.B, s_nb, s_rows, s_off);
-  if (it.b < 0) return;
-  const int b = it.b;
-  const int nb_old = it.nb - p.append;
-  const KT* K = static_cast<const KT*>(p.kcache) + static_cast<size_t>(b) * p.cap * d;
-  const KT* V = static_cast<const KT*>(p.vbuf) + static_cast<size_t>(b) * p.cap * d;
-  const KT* kn = static_cast<const KT*>(p.k_new) + static_cast<size_t>(b) * d;
+  LeanCursor cur;  // this CTA's segments
+  cur.init(blockIdx.x, p.B, s_q, s_plan);
+  SplitItem it;
+  while (cur.next(it, s_nb, s_q, s_soff)) {
+    const int b = it.b;
+    const int nb_old = it.nb - p.append;
+    const KT* K = static_cast<const KT*>(p.kcache) + static_cast<size_t>(b) * p.cap * d;
+    const KT* V = static_cast<const KT*>(p.vbuf) + static_cast<size_t>(b) * p.cap * d;
+    const KT* kn = static_cast<const KT*>(p.k_new) + static_cast<size_t>(b) * d;
 
-  for (int i = tid; i < d; i += blockDim.x) q_s[i] = p.q[static_cast<size_t>(b) * d + i];
-  const int nacc = VARIANT_A ? d : H * d;
-  for (int i = tid; i < nacc; i += blockDim.x) acc[i] = 0.f;
-  for (int h = tid; h < H; h += blockDim.x) {
-    mref[h] = -INFINITY;
-    lsum[h] = 0.f;
-  }
-  __syncthreads();
-
-  for (int r_lo = it.row0; r_lo < it.row1; r_lo += kSimtRows) {
-    const int nvalid = min(kSimtRows, it.row1 - r_lo);
-    for (int i = tid; i < kSimtRows * d; i += blockDim.x) {
-      const int row = i / d, col = i % d;
-      const int r = r_lo + row;
-      KT kv = from_f<KT>(0.f), vv = from_f<KT>(0.f);
-      if (row < nvalid) {
-        if (!VARIANT_A && p.append && r == nb_old) {
-          kv = kn[col];
-          static_cast<KT*>(p.kcache)[(static_cast<size_t>(b) * p.cap + r) * d + col] = kv;
-        } else {
-          kv = K[static_cast<size_t>(r) * d + col];
-        }
-        if (VARIANT_A) vv = V[static_cast<size_t>(r) * d + col];
-      }
-      ks[i] = kv;
-      if (VARIANT_A) vs[i] = vv;
-    }
-    __syncthreads();
-    // scores: warp w takes row w of the tile, every head
-    if (warp < kSimtRows) {
-      for (int h = 0; h < H; ++h) {
-        float s = 0.f;
-        for (int j = lane; j < d_h; j += 32) s = fmaf(q_s[h * d_h + j], to_f<KT>(ks[warp * d + h * d_h + j]), s);
-        s = warp_sum(s);
-        if (lane == 0) sc[h * kSimtRows + warp] = (warp < nvalid) ? s * p.scale_log2 : -INFINITY;
-      }
-    }
-    __syncthreads();
-    // exact online softmax update per head
+    for (int i = tid; i < d; i += blockDim.x) q_s[i] = p.q[static_cast<size_t>(b) * d + i];
+    const int nacc = VARIANT_A ? d : H * d;
+    for (int i = tid; i < nacc; i += blockDim.x) acc[i] = 0.f;
     for (int h = tid; h < H; h += blockDim.x) {
-      float mt = -INFINITY;
-      for (int t = 0; t < kSimtRows; ++t) mt = fmaxf(mt, sc[h * kSimtRows + t]);
-      const float mn = fmaxf(mref[h], mt);
-      const float a = exp2f(mref[h] - mn);
-      float ls = 0.f;
-      for (int t = 0; t < kSimtRows; ++t) {
-        const float pv = (t < nvalid) ? exp2f(sc[h * kSimtRows + t] - mn) : 0.f;
-        pm[h * kSimtRows + t] = pv;
-        ls += pv;
-      }
-      lsum[h] = lsum[h] * a + ls;
-      mref[h] = mn;
-      alph[h] = a;
+      mref[h] = -INFINITY;
+      lsum[h] = 0.f;
     }
     __syncthreads();
-    if (VARIANT_A) {
-      for (int col = tid; col < d; col += blockDim.x) {
-        const int h = col / d_h;
-        float x = acc[col] * alph[h];
-        for (int t = 0; t < kSimtRows; ++t) x = fmaf(pm[h * kSimtRows + t], to_f<KT>(vs[t * d + col]), x);
-        acc[col] = x;
+
+    for (int r_lo = it.row0; r_lo < it.row1; r_lo += kSimtRows) {
+      const int nvalid = min(kSimtRows, it.row1 - r_lo);
+      for (int i = tid; i < kSimtRows * d; i += blockDim.x) {
+        const int row = i / d, col = i % d;
+        const int r = r_lo + row;
+        KT kv = from_f<KT>(0.f), vv = from_f<KT>(0.f);
+        if (row < nvalid) {
+          if (!VARIANT_A && p.append && r == nb_old) {
+            kv = kn[col];
+            static_cast<KT*>(p.kcache)[(static_cast<size_t>(b) * p.cap + r) * d + col] = kv;
+          } else {
+            kv = K[static_cast<size_t>(r) * d + col];
+          }
+          if (VARIANT_A) vv = V[static_cast<size_t>(r) * d + col];
+        }
+        ks[i] = kv;
+        if (VARIANT_A) vs[i] = vv;
       }
-    } else {
-      for (int i = tid; i < H * d; i += blockDim.x) {
-        const int h = i / d, col = i % d;
-        float x = acc[i] * alph[h];
-        for (int t = 0; t < kSimtRows; ++t) x = fmaf(pm[h * kSimtRows + t], to_f<KT>(ks[t * d + col]), x);
-        acc[i] = x;
+      __syncthreads();
+      // scores: warp w takes row w of the tile, every head
+      if (warp < kSimtRows) {
+        for (int h = 0; h < H; ++h) {
+          float s = 0.f;
+          for (int j = lane; j < d_h; j += 32) s = fmaf(q_s[h * d_h + j], to_f<KT>(ks[warp * d + h * d_h + j]), s);
+          s = warp_sum(s);
+          if (lane == 0) sc[h * kSimtRows + warp] = (warp < nvalid) ? s * p.scale_log2 : -INFINITY;
+        }
       }
+      __syncthreads();
+      // exact online softmax update per head
+      for (int h = tid; h < H; h += blockDim.x) {
+        float mt = -INFINITY;
+        for (int t = 0; t < kSimtRows; ++t) mt = fmaxf(mt, sc[h * kSimtRows + t]);
+        const float mn = fmaxf(mref[h], mt);
+        const float a = exp2f(mref[h] - mn);
+        float ls = 0.f;
+        for (int t = 0; t < kSimtRows; ++t) {
+          const float pv = (t < nvalid) ? exp2f(sc[h * kSimtRows + t] - mn) : 0.f;
+          pm[h * kSimtRows + t] = pv;
+          ls += pv;
+        }
+        lsum[h] = lsum[h] * a + ls;
+        mref[h] = mn;
+        alph[h] = a;
+      }
+      __syncthreads();
+      if (VARIANT_A) {
+        for (int col = tid; col < d; col += blockDim.x) {
+          const int h = col / d_h;
+          float x = acc[col] * alph[h];
+          for (int t = 0; t < kSimtRows; ++t) x = fmaf(pm[h * kSimtRows + t], to_f<KT>(vs[t * d + col]), x);
+          acc[col] = x;
+        }
+      } else {
+        for (int i = tid; i < H * d; i += blockDim.x) {
+          const int h = i / d, col = i % d;
+          float x = acc[i] * alph[h];
+          for (int t = 0; t < kSimtRows; ++t) x = fmaf(pm[h * kSimtRows + t], to_f<KT>(ks[t * d + col]), x);
+          acc[i] = x;
+        }
+      }
+      __syncthreads();
     }
-    __syncthreads();
-  }
-  const size_t item = blockIdx.x;
-  for (int i = tid; i < nacc; i += blockDim.x) p.ws_U[item * nacc + i] = acc[i];
-  for (int h = tid; h < H; h += blockDim.x) {
-    p.ws_m[item * H + h] = mref[h];
-    p.ws_l[item * H + h] = lsum[h];
+    const size_t slot = static_cast<size_t>(it.slot);
+    for (int i = tid; i < nacc; i += blockDim.x) p.ws_U[slot * nacc + i] = acc[i];
+    for (int h = tid; h < H; h += blockDim.x) {
+      p.ws_m[slot * H + h] = mref[h];
+      p.ws_l[slot * H + h] = lsum[h];
+    }
+    __syncthreads();  // the next segment reuses q, the accumulator and the softmax state
   }
 }
 
@@ -280,7 +285,7 @@ SimtParams make_simt(const DecodeArgs& a, const SplitWorkspace& ws, bool variant
   const int app = a.k_new != nullptr ? 1 : 0;
   p.append = variant_a ? 0 : app;
   p.attend_add = app;
-  p.n_slots = ws.max_items;
+  p.n_slots = num_sms();
   p.min_rows = max(16, 8 * a.H);
   p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(a.d / a.H));
   return p;
@@ -294,7 +299,7 @@ cudaError_t launch_simt(const DecodeArgs& a, const SplitWorkspace& ws, cudaStrea
   auto kern = (a.dtype == SLIM_BF16) ? decode_simt_kernel<__nv_bfloat16, VA> : decode_simt_kernel<float, VA>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  kern<<<ws.max_items, 256, smem, st>>>(p);
+  kern<<<p.n_slots, 256, smem, st>>>(p);
   return cudaGetLastError();
 }
 }  // namespace

@@ -2,30 +2,34 @@
 //
 // Ordering (b) (Slim Attention article, section "K-Cache is All You Need",
 // second generation-phase option, with W_KV = W_K^(-1)·W_V): for sequence b
-// and head h, the chunk partials (m_c, l_c, U_c) combine by the log-sum-exp
-// rule into  ū = Σ_c 2^(m_c - M) U_c / Σ_c 2^(m_c - M) l_c,  M = max_c m_c,
+// and head h, the partials (m_c, l_c, U_c) of the sequence's segments combine
+// by the log-sum-exp rule into
+//     ū = Σ_c 2^(m_c - M) U_c / Σ_c 2^(m_c - M) l_c,   M = max_c m_c,
 // and the head output is  o[b, h-cols] = ū · W_KV[:, h-cols].
 //
-// The merge is small and latency-bound, so it is laid out to wait for memory
-// as few times as possible. Grid (H, NDB), clusters of NDB CTAs along y; CTA
-// (h, r) owns head h and the d-block r (DB = d / NDB columns).
-//   * Before the split kernel's results are awaited, its W_KV block (DB rows of
-//     the head-h columns; a parameter, not a result) is requested by TMA.
-//   * Then every thread issues all its loads at once: its items' slice of U
-//     (16-byte loads, two rounds of eight in flight), and the items' m and l.
-//   * One warp per sequence turns m, l into merge weights; each thread scales
-//     its U rows and adds them, per sequence, into ū in shared memory.
-//   * o_r[b, :] = ū[b, block] · W_KV[block, h-cols] on mma.sync (bf16 W_KV; ū
-//     as a bf16 high + low pair, fp32 accumulation) or fp32 FMAs (fp32 W_KV).
-//   * Each CTA pushes its product into the owner CTA of every output element
-//     (distributed shared memory) and signals the owner's mbarrier; owners add
-//     the NDB products in a fixed order and write o.
-// The kernel is a programmatic dependent of the split kernel.
+// Three kernels, chosen by shape (launch_reduce_b):
+//   * merge_lean_kernel  one CTA per (head, sequence): d_h = 64, d <= 1280 and
+//     B·H CTAs in one wave; the head slice of W_KV is held whole in shared memory.
+//   * merge_proj_kernel  bf16 W_KV with d_h = 64 or 128, any batch: one CTA per
+//     (head, block of d rows), all CTAs in one wave, clusters along the blocks.
+//     The partial rows are read with many loads in flight per thread, W_KV
+//     through a ring of TMA tiles; the projection runs on mma.sync; the blocks'
+//     products are summed in a fixed order through distributed shared memory.
+//   * merge_b_kernel     the same decomposition on the CUDA cores, for fp32
+//     W_KV (and bf16 shapes the other two do not take).
+// Each is a programmatic dependent of the split kernel: what does not depend
+// on the split's results (barriers, the first W_KV tiles) happens before the
+// wait.
 //
 // Ordering (a) needs only the merge (its partials are already softmax·V).
 #include <cuda_bf16.h>
 
 #include <algorithm>
+#include <map>
+#include <mutex>
+#include <tuple>
+#include <type_traits>
+#include <utility>
 
 #include "ptx.cuh"
 
@@ -41,14 +45,11 @@ struct MergeBParams {
   int32_t* status;
   int B, d, H, ndb, max_items;
   int b_begin, nb;  // sequences of this launch
-  int use_mma;      // bf16 W_KV, d_h a multiple of 64: swizzled W block, tensor-core projection
-  int cap_ranges;   // the split fills (nearly) every work slot: item runs sized by the capacity
 };
 
 constexpr int kMergeThreads = 256;
 constexpr int kMergeWarps = kMergeThreads / 32;
 constexpr int kMergeMaxSeqs = 128;  // sequences per launch (MMA rows)
-constexpr int kMergeMaxTiles = 8;   // 16x8 output tiles per warp
 constexpr int kMergeRound = 8;      // 16-byte loads in flight per thread and round
 
 struct MergeSmem {
@@ -105,12 +106,11 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
     mbar_init(wbar, 1);
     fence_barrier_init();
     tma_prefetch_desc(&wmap);
-    const int groups = p.use_mma ? d_h / 64 : 1, gcols = p.use_mma ? 64 : d_h, yrows = min(DB, 256);
+    const int yrows = min(DB, 256);
     mbar_arrive_expect_tx(wbar, static_cast<uint32_t>(DB) * d_h * sizeof(WT));
-    for (int g = 0; g < groups; ++g)
-      for (int y = 0; y < DB; y += yrows)
-        tma_load_2d(msm + L.w + static_cast<size_t>(g * DB + y) * gcols * sizeof(WT), &wmap, h * d_h + g * 64, c0 + y,
-                    wbar, l2_policy_evict_last());
+    for (int y = 0; y < DB; y += yrows)
+      tma_load_2d(msm + L.w + static_cast<size_t>(y) * d_h * sizeof(WT), &wmap, h * d_h, c0 + y, wbar,
+                  l2_policy_evict_last());
   }
   for (int i = tid; i < Bp * ubs; i += kMergeThreads) ub[i] = 0.f;
   if (p.ndb > 1) cluster_arrive_relaxed();
@@ -120,19 +120,14 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
   // ---- every load at once: this thread's U slices, then the work list and m, l
   const int it0 = b0 == 0 ? 0 : __ldcg(p.meta + 1 + b0);
   const int ncap = p.max_items - it0;
-  // Thread (cg, ig) takes columns 4cg.. of a contiguous run of items (runs of one sequence
-  // then add up in registers). When the split fills nearly every work slot the runs are sized
-  // by the capacity, so the first loads need no read of the work list; otherwise they are
-  // balanced over the items the split kernel produced.
+  // Thread (cg, ig) takes columns 4cg.. of a contiguous run of slots (runs of one sequence
+  // then add up in registers), balanced over the slots the split kernel produced.
   const int C4 = DB / 4, IG = kMergeThreads / C4;
   const int cg = tid % C4, ig = tid < IG * C4 ? tid / C4 : IG;
-  int ipt = (ncap + IG - 1) / IG, n_real = ncap;
-  if (!p.cap_ranges) {
-    n_real = min(ncap, __ldcg(p.meta + 1 + b0 + nb) - it0);  // items of this launch's sequences
-    ipt = (n_real + IG - 1) / IG;
-  }
+  const int n_real = min(ncap, __ldcg(p.meta + 1 + b0 + nb) - it0);  // slots of this launch's sequences
+  const int ipt = (n_real + IG - 1) / IG;
   const int i_beg = ig * ipt;
-  int i_end = ig < IG ? min(n_real, i_beg + ipt) : i_beg;
+  const int i_end = ig < IG ? min(n_real, i_beg + ipt) : i_beg;
   const float4* ubase = reinterpret_cast<const float4*>(p.U + (static_cast<size_t>(it0) * p.H + h) * p.d + c0) + cg;
   const size_t istride = static_cast<size_t>(p.H) * p.d / 4;  // float4 stride between items
   const int nrounds = (ipt + kMergeRound - 1) / kMergeRound;
@@ -145,7 +140,6 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
     }
   };
   load_round(bufA, 0);
-  if (p.cap_ranges) i_end = min(i_end, __ldcg(p.meta + 1 + b0 + nb) - it0);  // later rounds: real items only
   if (nrounds > 1) load_round(bufB, 1);
   for (int i = tid; i <= nb; i += kMergeThreads) s_off[i] = __ldcg(p.meta + 1 + b0 + i) - it0;
   for (int i = tid; i < ncap; i += kMergeThreads) {
@@ -219,41 +213,7 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
   if (!ok && tid == 0) mbar_wait(wbar, 0u, p.status);
 
   // ---- this CTA's product o_r[b, :] = ū[b, block] · W_KV[block, h-cols]
-  if (ok && p.use_mma && nb > 4) {
-    // 16x8 tiles: rows = sequences, columns = 8 of the head's d_h; ū = hi + lo in bf16
-    const int NT = d_h / 8, T = (Bp / 16) * NT;
-    const uint32_t wbase = smem_u32(msm + L.w);
-    const int g = lane >> 2, tq = lane & 3;
-#pragma unroll
-    for (int i = 0; i < kMergeMaxTiles; ++i) {
-      const int t = warp + kMergeWarps * i;
-      if (t >= T) break;
-      const int mt = t / NT, nt = t - mt * NT;
-      const int wb = nt >> 3, chunk = nt & 7;
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int ks = 0; ks < DB / 16; ++ks) {
-        const int row = ks * 16 + (lane & 15);
-        uint32_t b0f, b1f;
-        ldmatrix_x2_trans(wbase + (wb * DB + row) * 128 + ((chunk ^ (row & 7)) << 4), b0f, b1f);
-        const float* a = ub + (mt * 16 + g) * ubs + ks * 16 + 2 * tq;
-        const float2 xs[4] = {*reinterpret_cast<const float2*>(a), *reinterpret_cast<const float2*>(a + 8 * ubs),
-                              *reinterpret_cast<const float2*>(a + 8), *reinterpret_cast<const float2*>(a + 8 * ubs + 8)};
-        uint32_t ahi[4], alo[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const __nv_bfloat16 h0 = __float2bfloat16_rn(xs[e].x), h1 = __float2bfloat16_rn(xs[e].y);
-          ahi[e] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
-                   (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
-          alo[e] = pack_bf16x2(xs[e].x - __bfloat162float(h0), xs[e].y - __bfloat162float(h1));
-        }
-        mma_16816_bf16(acc, ahi, b0f, b1f);
-        mma_16816_bf16(acc, alo, b0f, b1f);
-      }
-      const int row = mt * 16 + g, col = nt * 8 + 2 * tq;
-      if (row < nb) *reinterpret_cast<float2*>(part + row * d_h + col) = make_float2(acc[0], acc[1]);
-      if (row + 8 < nb) *reinterpret_cast<float2*>(part + (row + 8) * d_h + col) = make_float2(acc[2], acc[3]);
-    }
-  } else if (ok) {
+  if (ok) {
     // FMAs: thread -> (sequence, 4 columns, one of S interleaved row subsets of the block),
     // the S partial sums (adjacent lanes) added with shuffles
     const WT* wsm = reinterpret_cast<const WT*>(msm + L.w);
@@ -269,19 +229,9 @@ __global__ void __launch_bounds__(kMergeThreads, 2)
         for (int c = cs; c < DB; c += S) {
           const float u = ub[bl * ubs + c];
           float w[4];
-          if (p.use_mma) {  // swizzled 64-column boxes of bf16
-            const int wb = j >> 6, jj = j & 63;
-            const uint8_t* rowp = msm + L.w + static_cast<size_t>(wb * DB + c) * 128;
-            const uint2 v = *reinterpret_cast<const uint2*>(rowp + ((((jj >> 3) ^ (c & 7)) << 4) | ((jj & 7) * 2)));
-            w[0] = bf16lo(v.x);
-            w[1] = bf16hi(v.x);
-            w[2] = bf16lo(v.y);
-            w[3] = bf16hi(v.y);
-          } else {
-            const WT* wr = wsm + static_cast<size_t>(c) * d_h + j;
+          const WT* wr = wsm + static_cast<size_t>(c) * d_h + j;
 #pragma unroll
-            for (int v = 0; v < 4; ++v) w[v] = static_cast<float>(wr[v]);
-          }
+          for (int v = 0; v < 4; ++v) w[v] = static_cast<float>(wr[v]);
           a.x = fmaf(u, w[0], a.x);
           a.y = fmaf(u, w[1], a.y);
           a.z = fmaf(u, w[2], a.z);
@@ -525,6 +475,286 @@ __global__ void __launch_bounds__(kLeanThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------- projection merge
+// bf16 W_KV, d_h = 64 DHB (DHB = 1 or 2), up to 16 MT sequences per launch. Grid (H, NDB),
+// clusters of NDB CTAs along y; CTA (h, r) owns head h and the rows [r·DB, (r+1)·DB) of W_KV,
+// DB = 256 VEC (VEC = 1, 2 or 4).
+//   * Before the split kernel's results are awaited: barriers, zeroed ū, and the first
+//     `ws` tiles of W_KV[block rows, head-h columns] (64 rows x 64 columns per TMA box,
+//     128-byte swizzle) requested into a ring of `ws` stages.
+//   * The slot range of the launch's sequences and, one warp per sequence, the merge weights
+//     from the slots' m and l.
+//   * ū[b, block] = Σ_c w_c U_c[block]: thread t owns the VEC columns VEC t ..; it loads its
+//     part of kProjDepth / VEC slots' rows at once (plain loads, all in flight together, no
+//     barrier) and adds them in slot order, so a sequence's sum is finished when its last slot
+//     has been added and the order of the additions is fixed.
+//   * o_r[b, :] = ū[b, block] · W_KV[block, h-cols] on mma.sync m16n8k16 (ū as a bf16 high and
+//     low part, fp32 accumulation), the W_KV tiles streamed through the ring.
+//   * The NDB products of an output element are pushed to one owner CTA and added there in a
+//     fixed order, so the result does not depend on timing.
+struct MergeProjParams {
+  const float* U;
+  const float* m;
+  const float* l;
+  const int32_t* meta;
+  float* out;
+  int32_t* lens;
+  int32_t* status;
+  int B, d, H, ndb, max_items;
+  int b_begin, nb;  // sequences of this launch (nb <= 16 MT)
+  int ws;           // W_KV ring stages
+};
+
+constexpr int kProjThreads = 256;
+constexpr int kProjWarps = kProjThreads / 32;
+constexpr int kProjWRows = 64;       // W_KV rows per ring stage
+constexpr int kProjMaxWStages = 16;  // W_KV ring stages at most
+constexpr int kProjDepth = 64;       // U floats in flight per thread
+
+struct ProjSmem {
+  uint32_t w, ub, ubs, wts, soff, part, recv, per, bars, total;
+};
+__host__ __device__ inline ProjSmem proj_smem_layout(int DB, int d_h, int nb, int ndb, int ws, int max_items) {
+  ProjSmem s;
+  uint32_t o = 0;
+  s.w = o;  // [ws][d_h / 64 boxes][64 rows][128 bytes], each stage a multiple of 1024 bytes
+  o += static_cast<uint32_t>(ws) * kProjWRows * d_h * 2u;
+  s.ubs = static_cast<uint32_t>(DB) + 8u;  // row stride of ū (floats): conflict-free fragment loads
+  s.ub = o;
+  o += up_to(static_cast<uint32_t>(nb), 16u) * s.ubs * 4u;
+  s.wts = o;
+  o += up_to(static_cast<uint32_t>(max_items), 4u) * 4u;
+  s.soff = o;
+  o += up_to(static_cast<uint32_t>(nb) + 1u, 4u) * 4u;
+  s.part = o;  // this CTA's product [nb][d_h]
+  o += static_cast<uint32_t>(nb) * d_h * 4u;
+  s.per = (static_cast<uint32_t>(nb) * d_h + ndb - 1u) / ndb;
+  s.recv = o;  // products pushed by the cluster's CTAs: [ndb][per]
+  o += static_cast<uint32_t>(ndb) * s.per * 4u;
+  o = up_to(o, 8u);
+  s.bars = o;
+  o += static_cast<uint32_t>(ws) * 8u;
+  s.total = o + 1024u;  // slack to align the base to 1024 bytes
+  return s;
+}
+
+// ū rows of the launch's sequences from their slots (see the kernel's comment); VEC columns per thread.
+template <int VEC>
+__device__ __forceinline__ void proj_merge_rows(const float* ubase, size_t ustride, int nrows, int s_beg,
+                                                const int* s_off, const float* wts, float* ub, int ubs, int tid) {
+  constexpr int D = kProjDepth / VEC;  // rows in flight
+  typedef typename std::conditional<VEC == 4, float4, typename std::conditional<VEC == 2, float2, float>::type>::type
+      VT;
+  float acc[VEC];
+#pragma unroll
+  for (int k = 0; k < VEC; ++k) acc[k] = 0.f;
+  int bl = 0;
+  const VT* src = reinterpret_cast<const VT*>(ubase) + tid;
+  const size_t vstride = ustride / VEC;
+  for (int c0 = 0; c0 < nrows; c0 += D) {
+    VT v[D];
+#pragma unroll
+    for (int u = 0; u < D; ++u) {
+      if (c0 + u < nrows) v[u] = __ldcg(src + static_cast<size_t>(c0 + u) * vstride);
+    }
+#pragma unroll
+    for (int u = 0; u < D; ++u) {
+      const int c = c0 + u;
+      if (c >= nrows) break;
+      while (s_beg + c >= s_off[bl + 1]) {  // the previous sequence is complete
+#pragma unroll
+        for (int k = 0; k < VEC; ++k) {
+          ub[bl * ubs + VEC * tid + k] = acc[k];
+          acc[k] = 0.f;
+        }
+        ++bl;
+      }
+      const float w = wts[c];
+      const float* x = reinterpret_cast<const float*>(&v[u]);
+#pragma unroll
+      for (int k = 0; k < VEC; ++k) acc[k] = fmaf(w, x[k], acc[k]);
+    }
+  }
+  if (nrows > 0) {
+#pragma unroll
+    for (int k = 0; k < VEC; ++k) ub[bl * ubs + VEC * tid + k] = acc[k];
+  }
+}
+
+template <int DHB, int MT>
+__global__ void __launch_bounds__(kProjThreads, 1)
+    merge_proj_kernel(const __grid_constant__ CUtensorMap wmap, const MergeProjParams p) {
+  extern __shared__ uint8_t psm_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(psm_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int DH = 64 * DHB;
+  constexpr int NT = DH / 8;                  // 8-column output tiles of a head
+  constexpr int TPW = MT * NT / kProjWarps;   // output tiles per warp
+  static_assert(TPW >= 1 && TPW * kProjWarps == MT * NT, "tiles must split evenly over the warps");
+  const int h = blockIdx.x, r = blockIdx.y;
+  const int DB = p.d / p.ndb, c0 = r * DB;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nb = p.nb, b0 = p.b_begin, WS = p.ws;
+  const ProjSmem L = proj_smem_layout(DB, DH, nb, p.ndb, WS, p.max_items);
+  uint8_t* wring = sm + L.w;
+  float* ub = reinterpret_cast<float*>(sm + L.ub);
+  float* wts = reinterpret_cast<float*>(sm + L.wts);
+  int* s_off = reinterpret_cast<int*>(sm + L.soff);
+  float* part = reinterpret_cast<float*>(sm + L.part);
+  float* recv = reinterpret_cast<float*>(sm + L.recv);
+  uint64_t* wfull = reinterpret_cast<uint64_t*>(sm + L.bars);
+  const int ubs = static_cast<int>(L.ubs), per = static_cast<int>(L.per);
+  const int nws = DB / kProjWRows;  // W_KV stages of this block
+  constexpr uint32_t kWStageBytes = kProjWRows * DH * 2u;
+
+  int w_issued = 0;  // thread 0 issues every W_KV copy
+  auto issue_w = [&](int st) {  // W_KV rows c0 + 64 st .., head-h columns, into ring stage st % WS
+    uint8_t* dst = wring + (st % WS) * kWStageBytes;
+    uint64_t* bar = &wfull[st % WS];
+    mbar_arrive_expect_tx(bar, kWStageBytes);
+#pragma unroll
+    for (int wb = 0; wb < DHB; ++wb)
+      tma_load_2d(dst + wb * kProjWRows * 128, &wmap, h * DH + wb * 64, c0 + st * kProjWRows, bar,
+                  l2_policy_evict_first());
+    ++w_issued;
+  };
+
+  // ---- before the split kernel's results exist
+  if (tid == 0) {
+    for (int s = 0; s < WS; ++s) mbar_init(&wfull[s], 1);
+    fence_barrier_init();
+    tma_prefetch_desc(&wmap);
+    for (int st = 0; st < min(WS, nws); ++st) issue_w(st);
+  }
+  const int Bp = (nb + 15) & ~15;
+  for (int i = tid; i < Bp * ubs; i += kProjThreads) ub[i] = 0.f;
+  if (p.ndb > 1) cluster_arrive_relaxed();
+  pdl_wait_primary();
+  pdl_launch_dependents();
+
+  // ---- slot ranges of the launch's sequences; the lengths advance once (CTA (0, 0))
+  for (int i = tid; i <= nb; i += kProjThreads) s_off[i] = __ldcg(p.meta + 1 + b0 + i);
+  if (h == 0 && r == 0)
+    for (int b = b0 + tid; b < b0 + nb; b += kProjThreads)
+      if (__ldcg(p.meta + 2 + p.B + b) & kSeqAppend) p.lens[b] += 1;
+  __syncthreads();
+  const int s_beg = s_off[0], nrows = s_off[nb] - s_beg;
+
+  // ---- merge weights 2^(m_c - M) / Σ_c' 2^(m_c' - M) l_c', one warp per sequence
+  for (int bl = warp; bl < nb; bl += kProjWarps) {
+    const int lo = s_off[bl], hi = s_off[bl + 1];
+    float M = -INFINITY;
+    for (int c = lo + lane; c < hi; c += 32) M = fmaxf(M, __ldcg(p.m + static_cast<size_t>(c) * p.H + h));
+    M = warp_max(M);
+    float S = 0.f;
+    for (int c = lo + lane; c < hi; c += 32) {
+      const float e = exp2f(__ldcg(p.m + static_cast<size_t>(c) * p.H + h) - M);
+      S = fmaf(e, __ldcg(p.l + static_cast<size_t>(c) * p.H + h), S);
+      wts[c - s_beg] = e;
+    }
+    S = warp_sum(S);
+    const float inv = S > 0.f ? 1.f / S : 0.f;
+    __syncwarp();
+    for (int c = lo + lane; c < hi; c += 32) wts[c - s_beg] *= inv;
+  }
+  __syncthreads();
+
+  // ---- ū[b, block] = Σ_c w_c U_c[block]
+  {
+    const float* ubase = p.U + (static_cast<size_t>(s_beg) * p.H + h) * p.d + c0;
+    const size_t ustride = static_cast<size_t>(p.H) * p.d;  // floats between slots
+    if (DB == 1024) proj_merge_rows<4>(ubase, ustride, nrows, s_beg, s_off, wts, ub, ubs, tid);
+    else if (DB == 512) proj_merge_rows<2>(ubase, ustride, nrows, s_beg, s_off, wts, ub, ubs, tid);
+    else proj_merge_rows<1>(ubase, ustride, nrows, s_beg, s_off, wts, ub, ubs, tid);
+  }
+  __syncthreads();
+
+  // ---- o_r = ū[:, block] · W_KV[block, h-cols] on mma.sync, W_KV through the ring
+  float acc[TPW][4];
+#pragma unroll
+  for (int i = 0; i < TPW; ++i)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[i][e] = 0.f;
+  const int g = lane >> 2, tq = lane & 3;
+  bool ok = true;
+  int w_done = 0;
+  for (int st = 0; st < nws; ++st) {
+    const bool got = mbar_wait(&wfull[st % WS], static_cast<uint32_t>(st / WS) & 1u, p.status);
+    if (got) {
+      const uint32_t wbase = smem_u32(wring + (st % WS) * kWStageBytes);
+#pragma unroll
+      for (int kk = 0; kk < kProjWRows / 16; ++kk) {
+        const int k0 = st * kProjWRows + kk * 16;  // column of ū
+        const int wrow = kk * 16 + (lane & 15);    // row within the stage
+        int mt_prev = -1;
+        uint32_t ahi[4], alo[4];
+#pragma unroll
+        for (int i = 0; i < TPW; ++i) {
+          const int t = warp + kProjWarps * i;
+          const int mt = t / NT, nt = t - mt * NT;
+          if (mt != mt_prev) {
+            mt_prev = mt;
+            const float* a = ub + (mt * 16 + g) * ubs + k0 + 2 * tq;
+            const float2 xs[4] = {*reinterpret_cast<const float2*>(a), *reinterpret_cast<const float2*>(a + 8 * ubs),
+                                  *reinterpret_cast<const float2*>(a + 8),
+                                  *reinterpret_cast<const float2*>(a + 8 * ubs + 8)};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const __nv_bfloat16 h0 = __float2bfloat16_rn(xs[e].x), h1 = __float2bfloat16_rn(xs[e].y);
+              ahi[e] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
+                       (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+              alo[e] = pack_bf16x2(xs[e].x - __bfloat162float(h0), xs[e].y - __bfloat162float(h1));
+            }
+          }
+          uint32_t b0f, b1f;
+          ldmatrix_x2_trans(wbase + ((nt >> 3) * kProjWRows + wrow) * 128 + (((nt & 7) ^ (wrow & 7)) << 4), b0f,
+                            b1f);
+          mma_16816_bf16(acc[i], ahi, b0f, b1f);
+          mma_16816_bf16(acc[i], alo, b0f, b1f);
+        }
+      }
+    }
+    ok = __syncthreads_and(got);  // every warp is done with the stage
+    if (!ok) break;
+    w_done = st + 1;
+    if (tid == 0 && st + WS < nws) issue_w(st + WS);
+  }
+  if (!ok && tid == 0) {
+    // copies still landing in this CTA's shared memory must complete before it exits
+    for (int st = w_done; st < w_issued; ++st)
+      mbar_wait(&wfull[st % WS], static_cast<uint32_t>(st / WS) & 1u, p.status);
+  }
+#pragma unroll
+  for (int i = 0; i < TPW; ++i) {
+    const int t = warp + kProjWarps * i;
+    const int mt = t / NT, nt = t - mt * NT;
+    const int row = mt * 16 + g, col = nt * 8 + 2 * tq;
+    if (row < nb) *reinterpret_cast<float2*>(part + row * DH + col) = make_float2(acc[i][0], acc[i][1]);
+    if (row + 8 < nb) *reinterpret_cast<float2*>(part + (row + 8) * DH + col) = make_float2(acc[i][2], acc[i][3]);
+  }
+  __syncthreads();
+
+  // ---- sum the NDB products: push each element to its owner CTA, then add in a fixed order
+  const int n_out = nb * DH;
+  if (p.ndb == 1) {
+    for (int e = tid; e < n_out; e += kProjThreads)
+      p.out[static_cast<size_t>(b0 + e / DH) * p.d + h * DH + e % DH] = ok ? part[e] : 0.f;
+    return;
+  }
+  cluster_wait();  // every CTA of the cluster is running
+  const uint32_t recv_base = smem_u32(recv);
+  for (int e = tid; e < n_out; e += kProjThreads)
+    st_cluster_f32(mapa_shared(recv_base + 4u * static_cast<uint32_t>(r * per + e / p.ndb), e % p.ndb),
+                   ok ? part[e] : 0.f);
+  cluster_sync();  // pushes visible; nobody touches a peer's shared memory after this
+  for (int s2 = tid; s2 < per; s2 += kProjThreads) {
+    const int e = s2 * p.ndb + r;
+    if (e >= n_out) break;
+    float a = 0.f;
+    for (int q = 0; q < p.ndb; ++q) a += recv[q * per + s2];
+    p.out[static_cast<size_t>(b0 + e / DH) * p.d + h * DH + e % DH] = a;
+  }
+}
+
 // ---------------------------------------------------------------------------- ordering (a) merge
 struct ReduceAParams {
   const float* O;
@@ -563,19 +793,17 @@ __global__ void __launch_bounds__(256) reduce_a_kernel(const ReduceAParams p) {
 namespace {
 
 struct MergeConfig {
-  int ndb, use_mma, nb_max;
+  int ndb, nb_max;
   size_t smem;
 };
 
-// NDB: the smallest of 1, 2, 4, 8 that gives at least one CTA per SM, preferring a
-// footprint that lets two CTAs share an SM; 16 (a non-portable cluster) only when no
-// smaller block fits.
+// CUDA-core merge: NDB the smallest of 1, 2, 4, 8 that gives at least one CTA per SM,
+// preferring a footprint that lets two CTAs share an SM; 16 (a non-portable cluster) only
+// when no smaller block fits.
 bool pick_merge(int B, int d, int H, int esz, int max_items, MergeConfig* c) {
   const int d_h = d / H;
-  const bool mma = esz == 2 && d_h % 64 == 0;
-  if (!mma && (d_h % 4 || (d_h * esz) % 16 || d_h > 256)) return false;
-  c->use_mma = mma ? 1 : 0;
-  c->nb_max = mma ? std::min(kMergeMaxSeqs, 16 * kMergeWarps * kMergeMaxTiles / (d_h / 8)) : kMergeMaxSeqs;
+  if (d_h % 4 || (d_h * esz) % 16 || d_h > 256) return false;
+  c->nb_max = kMergeMaxSeqs;
   const int nb = std::min(B, c->nb_max);
   const size_t half = static_cast<size_t>(max_smem_optin()) / 2 - 2048, full = static_cast<size_t>(max_smem_optin()) - 2048;
   // rank 3: enough CTAs and two per SM; 2: enough CTAs; 1: fits (the most blocks wins)
@@ -585,7 +813,7 @@ bool pick_merge(int B, int d, int H, int esz, int max_items, MergeConfig* c) {
     if (ndb == 16 && best != 0) break;
     if (d % ndb) break;
     const int DB = d / ndb;
-    if (DB % (mma ? 16 : 4) || (DB > 256 && DB % 256) || DB / 4 > kMergeThreads) continue;
+    if (DB % 4 || (DB > 256 && DB % 256) || DB / 4 > kMergeThreads) continue;
     const size_t sm = merge_smem_layout(DB, d_h, esz, nb, ndb, max_items).total;
     if (sm > full) continue;
     const bool enough = H * ndb >= num_sms();
@@ -601,6 +829,107 @@ bool pick_merge(int B, int d, int H, int esz, int max_items, MergeConfig* c) {
   c->ndb = best;
   c->smem = best_smem;
   return true;
+}
+
+struct ProjConfig {
+  int ndb, ws, nb_max;
+  uint32_t smem;
+};
+
+constexpr int kProjMaxSeqs = 64;  // sequences per launch: MT <= 4 tiles of 16
+
+template <int DHB, int MT>
+int proj_resident_clusters(int ndb, uint32_t smem, int H) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(H), static_cast<unsigned>(ndb), 1);
+  cfg.blockDim = dim3(kProjThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = static_cast<unsigned>(ndb);
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  auto kern = merge_proj_kernel<DHB, MT>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+int proj_resident(int dhb, int mt, int ndb, uint32_t smem, int H) {
+#define SLIM_PROJ_RES(D_, M_) \
+  if (dhb == D_ && mt == M_) return proj_resident_clusters<D_, M_>(ndb, smem, H);
+  SLIM_PROJ_RES(1, 1) SLIM_PROJ_RES(1, 2) SLIM_PROJ_RES(1, 3) SLIM_PROJ_RES(1, 4)
+  SLIM_PROJ_RES(2, 1) SLIM_PROJ_RES(2, 2) SLIM_PROJ_RES(2, 3) SLIM_PROJ_RES(2, 4)
+#undef SLIM_PROJ_RES
+  return 0;
+}
+
+// Projection merge for bf16 W_KV and d_h = 64 or 128. NDB (1..8, DB = d/NDB a multiple of 64
+// and at most 1024) is chosen so that the H x NDB CTAs run in one wave with as many CTAs as
+// possible (the fewest blocks on a tie); the U ring holds about 64 KB of rows in flight.
+bool pick_proj_uncached(int B, int d, int H, int max_items, ProjConfig* c) {
+  const int d_h = d / H;
+  if (d_h != 64 && d_h != 128) return false;
+  c->nb_max = kProjMaxSeqs;
+  const int nb = std::min(B, kProjMaxSeqs);
+  const int mt = (nb + 15) / 16;
+  const uint32_t optin = static_cast<uint32_t>(max_smem_optin());
+  int best = 0, best_ctas = -1, best_ws = 0;
+  uint32_t best_smem = 0;
+  for (int ndb = 1; ndb <= 8; ++ndb) {
+    if (d % ndb) continue;
+    const int DB = d / ndb;
+    if (DB != 256 && DB != 512 && DB != 1024) continue;
+    // as many W_KV stages as fit (the whole block when it does), at least two
+    int ws = std::min(kProjMaxWStages, DB / kProjWRows);
+    uint32_t sm = proj_smem_layout(DB, d_h, nb, ndb, ws, max_items).total;
+    while (sm > optin && ws > 2) sm = proj_smem_layout(DB, d_h, nb, ndb, --ws, max_items).total;
+    if (sm > optin) continue;
+    const int fit = proj_resident(d_h / 64, mt, ndb, sm, H);  // clusters resident at once
+    if (fit <= 0) continue;
+    const int score = H <= fit ? H * ndb : 0;  // CTAs, when all of them run in one wave
+    if (score > best_ctas) {
+      best = ndb;
+      best_ctas = score;
+      best_ws = ws;
+      best_smem = sm;
+    }
+  }
+  if (best == 0) return false;
+  c->ndb = best;
+  c->ws = best_ws;
+  c->smem = best_smem;
+  return true;
+}
+
+// pick_proj_uncached memoised per (device, shape): it queries the occupancy API.
+bool pick_proj(int B, int d, int H, int max_items, ProjConfig* c) {
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, int, int, int>, std::pair<bool, ProjConfig>> memo;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  const auto key = std::make_tuple(dev, B, d, H, max_items);
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = memo.find(key);
+  if (it == memo.end()) {
+    ProjConfig pc{};
+    const bool ok = pick_proj_uncached(B, d, H, max_items, &pc);
+    it = memo.emplace(key, std::make_pair(ok, pc)).first;
+  }
+  *c = it->second.second;
+  return it->second.first;
 }
 
 }  // namespace
@@ -661,26 +990,96 @@ cudaError_t launch_merge_lean(const DecodeArgs& a, const SplitWorkspace& ws, int
 
 }  // namespace
 
+namespace {
+
+template <int DHB, int MT>
+cudaError_t launch_proj_instance(const CUtensorMap& wmap, const MergeProjParams& p, uint32_t smem, bool pdl,
+                                 cudaStream_t st) {
+  auto kern = merge_proj_kernel<DHB, MT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(p.H), static_cast<unsigned>(p.ndb), 1);
+  cfg.blockDim = dim3(kProjThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = static_cast<unsigned>(p.ndb);
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kern, wmap, p);
+}
+
+cudaError_t launch_merge_proj(const DecodeArgs& a, const SplitWorkspace& ws, const ProjConfig& c, bool pdl,
+                              cudaStream_t st, int* launches) {
+  const int d_h = a.d / a.H, DB = a.d / c.ndb;
+  // W_KV as {d columns, d rows}, bf16; a box is 64 columns x 64 rows, 128-byte swizzled
+  CUtensorMap wmap;
+  const uint64_t dims[2] = {static_cast<uint64_t>(a.d), static_cast<uint64_t>(a.d)};
+  const uint64_t strides[1] = {static_cast<uint64_t>(a.d) * 2u};
+  const uint32_t box[2] = {64u, static_cast<uint32_t>(kProjWRows)};
+  if (!encode_tmap(&wmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.w_kv, dims, strides, box, true))
+    return cudaErrorInvalidValue;
+  for (int b0 = 0; b0 < a.B; b0 += c.nb_max) {
+    MergeProjParams p;
+    p.U = ws.U;
+    p.m = ws.m;
+    p.l = ws.l;
+    p.meta = ws.meta;
+    p.out = a.out;
+    p.lens = a.lens;
+    p.status = a.status;
+    p.B = a.B;
+    p.d = a.d;
+    p.H = a.H;
+    p.ndb = c.ndb;
+    p.max_items = ws.max_items;
+    p.b_begin = b0;
+    p.nb = std::min(c.nb_max, a.B - b0);
+    p.ws = c.ws;
+    const int mt = (p.nb + 15) / 16;
+    const uint32_t smem = proj_smem_layout(DB, d_h, p.nb, c.ndb, c.ws, ws.max_items).total;
+    const bool dep = pdl && b0 == 0;
+    cudaError_t e = cudaErrorNotSupported;
+#define SLIM_PROJ_CASE(D_, M_) \
+    if (d_h == 64 * D_ && mt == M_) e = launch_proj_instance<D_, M_>(wmap, p, smem, dep, st);
+    SLIM_PROJ_CASE(1, 1) SLIM_PROJ_CASE(1, 2) SLIM_PROJ_CASE(1, 3) SLIM_PROJ_CASE(1, 4)
+    SLIM_PROJ_CASE(2, 1) SLIM_PROJ_CASE(2, 2) SLIM_PROJ_CASE(2, 3) SLIM_PROJ_CASE(2, 4)
+#undef SLIM_PROJ_CASE
+    if (e != cudaSuccess) return e;
+    if (launches) ++*launches;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace
+
 cudaError_t launch_reduce_b(const DecodeArgs& a, const SplitWorkspace& ws, bool pdl, cudaStream_t st,
                             int* launches) {
   if (const int cap = lean_cap_items(a.B, a.d, a.H, a.dtype, ws.max_items))
     return launch_merge_lean(a, ws, cap, pdl, st, launches);
+  if (a.dtype == SLIM_BF16) {
+    ProjConfig pc;
+    if (pick_proj(a.B, a.d, a.H, ws.max_items, &pc)) return launch_merge_proj(a, ws, pc, pdl, st, launches);
+  }
   const int esz = a.dtype == SLIM_BF16 ? 2 : 4;
   const int d_h = a.d / a.H;
   MergeConfig c;
   if (!pick_merge(a.B, a.d, a.H, esz, ws.max_items, &c)) return cudaErrorNotSupported;
   const int DB = a.d / c.ndb;
-  // W_KV as {d columns, d rows}; a box is one 64-column swizzled group (MMA) or the head's d_h columns
+  // W_KV as {d columns, d rows}; a box is the head's d_h columns x up to 256 rows, dense
   CUtensorMap wmap;
   const uint64_t dims[2] = {static_cast<uint64_t>(a.d), static_cast<uint64_t>(a.d)};
   const uint64_t strides[1] = {static_cast<uint64_t>(a.d) * esz};
-  const uint32_t box[2] = {static_cast<uint32_t>(c.use_mma ? 64 : d_h), static_cast<uint32_t>(std::min(DB, 256))};
+  const uint32_t box[2] = {static_cast<uint32_t>(d_h), static_cast<uint32_t>(std::min(DB, 256))};
   if (!encode_tmap(&wmap, esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, a.w_kv,
-                   dims, strides, box, c.use_mma != 0))
+                   dims, strides, box, false))
     return cudaErrorInvalidValue;
-  // The tcgen05 split with single-CTA groups (CL = 1) plans one item per SM slot, so its
-  // items nearly fill the workspace capacity; other configurations leave most slots empty.
-  const bool cap_ranges = a.dtype == SLIM_BF16 && decode_b_tc_cluster(a.B, a.d, a.H) == 1;
   auto kern = (a.dtype == SLIM_BF16) ? merge_b_kernel<__nv_bfloat16> : merge_b_kernel<float>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(c.smem));
   if (e == cudaSuccess && c.ndb > 8) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
@@ -701,8 +1100,6 @@ cudaError_t launch_reduce_b(const DecodeArgs& a, const SplitWorkspace& ws, bool 
     p.max_items = ws.max_items;
     p.b_begin = b0;
     p.nb = std::min(c.nb_max, a.B - b0);
-    p.use_mma = c.use_mma;
-    p.cap_ranges = cap_ranges ? 1 : 0;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(a.H), static_cast<unsigned>(c.ndb), 1);
     cfg.blockDim = dim3(kMergeThreads, 1, 1);

@@ -122,7 +122,9 @@ struct WsLayout {
 
 WsLayout ws_layout(int dtype, int B, int d, int H, int64_t cap, int variant) {
   WsLayout w{};
-  const int items = std::max(num_sms(), B);
+  // partial slots: a split kernel runs at most num_sms() work groups, and a group's contiguous share
+  // of the rows adds one slot per sequence boundary inside it
+  const int items = num_sms() + B;
   w.max_items = items;
   const bool need_b = variant != SLIM_VARIANT_A;
   const bool need_a = variant != SLIM_VARIANT_B;
@@ -367,6 +369,41 @@ int slim_decode_step(const float* q, const void* k_new, void* Kcache, int32_t* l
     if (!decode_a_supported(dtype, B, d, H)) return SLIM_EUNSUPPORTED;
     e = launch_decode_a(a, ws, st, &launches);
   }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return e == cudaErrorNotSupported ? SLIM_EUNSUPPORTED : SLIM_ECUDA;
+  }
+  g_last_launches = launches;
+  return SLIM_OK;
+}
+
+size_t slim_mha_decode_workspace_bytes(int dtype, int B, int d, int H, int64_t cap) {
+  if (!valid_dims(dtype, B, d, H, cap) || dtype != SLIM_BF16 || !decode_kv_supported(B, d, H, cap)) return 0;
+  const size_t slots = kv_ws_slots(B, d);
+  const int hg = d / 256;
+  return up(slots * 256 * 4) + 2 * up(slots * 4 * 4) + up(meta_ints(B * hg) * 4);
+}
+
+int slim_mha_decode_step(const float* q, const void* k_new, const void* v_new, void* Kcache, void* Vcache,
+                         int32_t* lens, int dtype, int B, int d, int H, int64_t cap, float* out, void* workspace,
+                         size_t ws_bytes, int32_t* dev_status, void* stream) {
+  if (!q || !Kcache || !Vcache || !lens || !out || !dev_status || (!k_new != !v_new)) return SLIM_EINVAL;
+  if (!valid_dims(dtype, B, d, H, cap)) return SLIM_EINVAL;
+  if (!aligned(q, 16) || !aligned(Kcache, 16) || !aligned(Vcache, 16) || (k_new && !aligned(k_new, 16)) ||
+      (v_new && !aligned(v_new, 16)))
+    return SLIM_EINVAL;
+  if (dtype != SLIM_BF16 || !decode_kv_supported(B, d, H, cap)) return SLIM_EUNSUPPORTED;
+  const size_t need = slim_mha_decode_workspace_bytes(dtype, B, d, H, cap);
+  if (!workspace || !aligned(workspace, kAlign) || ws_bytes < need) return SLIM_EWORKSPACE;
+  const size_t slots = kv_ws_slots(B, d);
+  char* w = static_cast<char*>(workspace);
+  float* wsO = reinterpret_cast<float*>(w);
+  float* wsm = reinterpret_cast<float*>(w + up(slots * 256 * 4));
+  float* wsl = reinterpret_cast<float*>(w + up(slots * 256 * 4) + up(slots * 4 * 4));
+  int32_t* meta = reinterpret_cast<int32_t*>(w + up(slots * 256 * 4) + 2 * up(slots * 4 * 4));
+  int launches = 0;
+  const cudaError_t e = launch_decode_kv(q, k_new, v_new, Kcache, Vcache, lens, B, d, H, cap, out, wsO, wsm, wsl,
+                                         meta, dev_status, static_cast<cudaStream_t>(stream), &launches);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return e == cudaErrorNotSupported ? SLIM_EUNSUPPORTED : SLIM_ECUDA;

@@ -14,18 +14,17 @@ namespace slim {
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
 
 // Work-list metadata written by the split kernel for the merge kernel:
-//   meta[0]          total number of work items
-//   meta[1 + b]      first item of sequence b (b = 0..B), meta[1 + B] = total
+//   meta[0]          total number of partial slots
+//   meta[1 + b]      first slot of sequence b (b = 0..B), meta[1 + B] = total
 //   meta[2 + B + b]  flags of sequence b (kSeqAppend: lens[b] must advance by one)
-//   meta[2 + 2B]     chunk length the plan chose (the next plan's first candidate)
 constexpr int kSeqAppend = 1;
-__host__ __device__ inline size_t meta_ints(int B) { return static_cast<size_t>(2 * B + 3); }
+__host__ __device__ inline size_t meta_ints(int B) { return static_cast<size_t>(2 * B + 2); }
 
 // Scratch of the split-T orderings, carved from the caller's workspace.
 struct SplitWorkspace {
-  float* U;      // (b): [items][H][d] unnormalised softmax·K rows;  (a): [items][d] softmax·V
-  float* m;      // [items][H] running max (log2 domain)
-  float* l;      // [items][H] softmax denominators relative to m
+  float* U;      // (b): [slots][H][d] unnormalised softmax·K rows;  (a): [slots][d] softmax·V
+  float* m;      // [slots][H] running max (log2 domain)
+  float* l;      // [slots][H] softmax denominators relative to m
   int32_t* meta; // meta_ints(B)
   void* vbuf;    // (a) only: [B][cap][d] materialised V = K·W_KV
   void* qstage;  // staging for slim_decode_step_host: q, k_new, out
@@ -42,13 +41,6 @@ struct DecodeArgs {
   int64_t cap;
   float* out;
   int32_t* status;
-};
-
-// Split decomposition of the attended rows into work items; computed the
-// same way on the device by every CTA of a split kernel.
-struct SplitPlan {
-  int n_slots;   // clusters (work slots) launched
-  int min_rows;  // smallest chunk worth its partial write
 };
 
 // ---- launchers (return cudaError_t of the launch) ----
@@ -77,6 +69,13 @@ cudaError_t launch_rows_gemm_any(const void* A, const void* W, void* Y, const in
                                  int* launches);
 cudaError_t launch_rows_gemm(const void* A, const void* W, void* Y, const int32_t* lens, int rows_extra, int dtype,
                              int B, int d, int64_t cap, cudaStream_t st, int* launches);
+
+// Standard MHA decode over explicit K and V caches (the comparison baseline), bf16.
+bool decode_kv_supported(int B, int d, int H, int64_t cap);
+size_t kv_ws_slots(int B, int d);  // partial slots its workspace needs
+cudaError_t launch_decode_kv(const float* q, const void* k_new, const void* v_new, void* kcache, void* vcache,
+                             int32_t* lens, int B, int d, int H, int64_t cap, float* out, float* wsO, float* wsm,
+                             float* wsl, int32_t* meta, int32_t* status, cudaStream_t st, int* launches);
 
 // Tensor map encoding through the driver entry point (no link-time libcuda dependency).
 bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,

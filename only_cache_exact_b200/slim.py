@@ -28,6 +28,7 @@ EXPORTS = [
     "slim_prefill_k", "slim_decode_workspace_bytes", "slim_decode_step", "slim_decode_step_host", "slim_tune",
     "slim_tune_record", "slim_select_variant", "slim_tune_clear", "slim_strerror", "slim_last_launch_count",
     "slim_version", "slim_timing_enable", "slim_timing_read", "slim_decode_step_noalloc",
+    "slim_mha_decode_workspace_bytes", "slim_mha_decode_step",
 ]
 
 _vp, _i32, _i64, _sz, _f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
@@ -50,6 +51,9 @@ _SIGS = {
     "slim_timing_read": (_i32, [_vp, _i32]),
     "slim_decode_step_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i64, _i32, _i64, _vp, _vp,
                                         _vp]),
+    "slim_mha_decode_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i64]),
+    "slim_mha_decode_step": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i64, _vp, _vp, _sz, _vp,
+                                    _vp]),
 }
 SLIM_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 for _name, (_res, _args) in _SIGS.items():
@@ -152,6 +156,40 @@ def slim_decode_step_noalloc(q: torch.Tensor, k_new, Kcache: torch.Tensor, lens:
     _check(_lib.slim_decode_step_noalloc(_ptr(q), _ptr(k_new), _ptr(Kcache), _ptr(lens), _ptr(W_KV),
                                          _DT[Kcache.dtype], B, d, H, cap, variant, t_hint, _ptr(out), _ptr(status),
                                          _stream(stream)), "slim_decode_step_noalloc")
+
+
+def slim_mha_decode_workspace_bytes(dtype: int, B: int, d: int, H: int, cap: int) -> int:
+    return int(_lib.slim_mha_decode_workspace_bytes(dtype, B, d, H, cap))
+
+
+def alloc_mha_workspace(dtype: int, B: int, d: int, H: int, cap: int, device=None) -> torch.Tensor:
+    """Caller-owned scratch for slim_mha_decode_step."""
+    n = slim_mha_decode_workspace_bytes(dtype, B, d, H, cap)
+    if n == 0:
+        raise SlimError(SLIM_EUNSUPPORTED, "slim_mha_decode_workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device or torch.device("cuda"))
+
+
+def slim_mha_decode_step(q: torch.Tensor, k_new, v_new, Kcache: torch.Tensor, Vcache: torch.Tensor,
+                         lens: torch.Tensor, H: int, out: torch.Tensor, workspace: torch.Tensor, status: torch.Tensor,
+                         stream=None) -> None:
+    """Standard MHA generation step over explicit K and V caches [B][cap][d] (the comparison baseline)."""
+    for t, nm in ((q, "q"), (Kcache, "Kcache"), (Vcache, "Vcache"), (lens, "lens"), (out, "out"),
+                  (workspace, "workspace"), (status, "status")):
+        _cuda(t, nm)
+    B, cap, d = Kcache.shape
+    if Vcache.shape != Kcache.shape or Vcache.dtype != Kcache.dtype:
+        raise ValueError("Vcache must match Kcache")
+    if q.shape != (B, d) or out.shape != (B, d) or q.dtype != torch.float32 or out.dtype != torch.float32:
+        raise ValueError("q/out must be float32 [B][d]")
+    for t, nm in ((k_new, "k_new"), (v_new, "v_new")):
+        if t is not None:
+            _cuda(t, nm)
+            if t.shape != (B, d) or t.dtype != Kcache.dtype:
+                raise ValueError(f"{nm} must be [B][d] in the cache dtype")
+    _check(_lib.slim_mha_decode_step(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(Kcache), _ptr(Vcache), _ptr(lens),
+                                     _DT[Kcache.dtype], B, d, H, cap, _ptr(out), _ptr(workspace), workspace.numel(),
+                                     _ptr(status), _stream(stream)), "slim_mha_decode_step")
 
 
 def slim_decode_step_host(q_host: torch.Tensor, k_new_host, Kcache: torch.Tensor, lens: torch.Tensor,
