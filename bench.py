@@ -585,6 +585,27 @@ def run_sweep(S, dev):
         tot += e0.elapsed_time(e1)
     ms_p = tot / reps
     prefill = {"rows": chunk, "d": d, "ms": ms_p, "tflops": 2.0 * chunk * d * d / ms_p / 1e9}
+    # the prompt's attention output over the K-only cache: V = K·W_KV once, then causal attention
+    Qp = synth.make_tokens_device(chunk, d, 7, 0, "bf16", part=2, device=dev).view(1, chunk, d)
+    outp = torch.empty(1, chunk, d, dtype=torch.float32, device=dev)
+    wsp = torch.empty(S.slim_prefill_attention_workspace_bytes(S.SLIM_BF16, B, d, H, cap), dtype=torch.uint8,
+                      device=dev)
+    for _ in range(2):
+        S.slim_prefill_attention(Qp, K, lens, W_KV, H, outp, wsp, status)
+    torch.cuda.synchronize()
+    tot = 0.0
+    for _ in range(reps):
+        torch.cuda._sleep(int(5e6))
+        e0.record()
+        S.slim_prefill_attention(Qp, K, lens, W_KV, H, outp, wsp, status)
+        e1.record()
+        e1.synchronize()
+        tot += e0.elapsed_time(e1)
+    ms_att = tot / reps
+    att_flops = 2.0 * chunk * chunk * d + 2.0 * chunk * d * d  # causal QK^T and PV, plus V = K·W_KV
+    prefill["attention"] = {"queries": chunk, "ms": ms_att, "tflops": att_flops / ms_att / 1e9,
+                            "flops_note": "2·n²·d (causal QK^T and PV) + 2·n·d² (V = K·W_KV)"}
+    del wsp, outp
     for r0 in range(chunk, cap, chunk):
         Xr = synth.make_tokens_device(chunk, d, 1000 + r0 // chunk, 0, "bf16", device=dev).view(1, chunk, d)
         S.slim_prefill_k(Xr, W_K, K, lens, status)

@@ -165,6 +165,32 @@ int slim_decode_step_noalloc(const float* q, const void* k_new, void* Kcache, in
                              int32_t* dev_status, void* stream);
 
 /*
+ * slim_prefill_attention — prompt phase: the attention output of the n prompt
+ * tokens of every sequence, over the K-only cache. Source: section "K-Cache is
+ * All You Need", prompt phase (queries and keys of all prompt tokens in
+ * parallel, only K cached, values from K through W_KV). Call it after
+ * slim_prefill_k has appended the prompt's keys: the queries are those of the
+ * last n cached rows, query j of sequence b at position p = lens[b] - n + j,
+ * and it attends causally over rows 0..p (its own key included):
+ *     out[b][j][h-cols] = softmax(q_h·K_h[0..p]^T/sqrt(d_h)) · V_h[0..p],
+ * V = K·W_KV, computed once for the cached rows into the workspace (ordering
+ * (a): every query reuses it), then flash-attention over Q, K and V.
+ *
+ *   Q        [B][n][d] bf16            the prompt's queries (device, read)
+ *   Kcache   [B][cap][d] bf16          (device, read)
+ *   lens     int32[B]                  (device, read; not changed)
+ *   W_KV     [d][d] bf16
+ *   dtype    SLIM_BF16 only; d % 256 == 0, d_h = d/H of 64 or 128
+ *   out      float[B][n][d]            (device, written)
+ *   workspace >= slim_prefill_attention_workspace_bytes(...), 256-byte aligned
+ *   dev_status  SLIM_DEV_BADLEN if lens[b] < n or lens[b] > cap (sequence skipped)
+ */
+size_t slim_prefill_attention_workspace_bytes(int dtype, int B, int d, int H, int64_t cap);
+int slim_prefill_attention(const void* Q, const void* Kcache, const int32_t* lens, const void* W_KV, int dtype,
+                           int B, int n, int d, int H, int64_t cap, float* out, void* workspace, size_t ws_bytes,
+                           int32_t* dev_status, void* stream);
+
+/*
  * slim_mha_decode_step — the standard multi-head attention generation step
  * over explicit K and V caches, the step Slim attention rewrites: for every
  * sequence b and head h, o[b, h-cols] = softmax(q_h·K_h^T/sqrt(d_h))·V_h.
@@ -235,6 +261,20 @@ int slim_timing_enable(int n);
  * elapsed milliseconds of pair i into ms[i] for i < min(n, pairs recorded)
  * and returns that count (negative SLIM_E* on error). */
 int slim_timing_read(float* ms, int n);
+
+/*
+ * slim_debug_stall_next — test hook for the failure path. The next
+ * slim_decode_step on this host thread that runs the tcgen05 split kernel
+ * (ordering (b), bf16 cache) makes that kernel's MMA warp wait on a barrier
+ * that nothing completes, with every wait of that kernel limited to wait_ns
+ * nanoseconds (1000 <= wait_ns <= 1e9) instead of the usual second. The
+ * kernel then ORs SLIM_DEV_TIMEOUT into *dev_status, lets every copy it
+ * issued land, frees its tensor memory and returns; that step's output and
+ * the lengths it advances are not meaningful, the cache is not corrupted and
+ * the context stays usable. Returns SLIM_OK, or SLIM_EINVAL for wait_ns out
+ * of range. Host-side only.
+ */
+int slim_debug_stall_next(int64_t wait_ns);
 
 /* slim_version — ABI version (major*100 + minor). */
 int slim_version(void);

@@ -79,6 +79,8 @@ struct DecodeTCParams {
   int min_rows;
   uint32_t tmem_cols;
   float scale_log2;
+  uint64_t wait_ns;  // limit of every wait (kWaitLimitNs unless a test shortens it)
+  int stall;         // test hook: the MMA warp first waits on a barrier nothing completes
 };
 
 // Shared-memory carve-up, identical on host and device.
@@ -99,7 +101,7 @@ __host__ __device__ inline TCSmem tc_smem_layout(int CL, int TT, int d, int stag
   o += dS * 4u;
   o = (o + 7u) & ~7u;
   s.bar_off = o;
-  o += (5u * stages + 2u) * 8u;
+  o += (5u * stages + 3u) * 8u;
   s.slot_off = o;
   o += 16u;
   s.plan_off = o;  // s_nb [B + 1], s_q [B + 1], s_soff [B + 1], s_plan [2]
@@ -182,6 +184,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
   uint64_t* corr = bars + 4 * stages;          // accumulator corrected for this tile's new maxima
   uint64_t* accfull = bars + 5 * stages;       // last MMA of a segment completed
   uint64_t* accempty = bars + 5 * stages + 1;  // epilogue finished reading the accumulator
+  uint64_t* stallbar = bars + 5 * stages + 2;  // test hook: never completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.slot_off);
   int* s_nb = reinterpret_cast<int*>(smem + L.plan_off);
   unsigned* s_q = reinterpret_cast<unsigned*>(s_nb + (p.B + 1));
@@ -210,6 +213,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
       }
       mbar_init(accfull, 1);
       mbar_init(accempty, 4);
+      mbar_init(stallbar, 1);
       fence_barrier_init();
     }
     __syncwarp();
@@ -249,7 +253,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
         for (int t = 0; t < nt; ++t, ++g) {
           const int s = g % stages;
           const uint32_t ph = static_cast<uint32_t>(g / stages) & 1u;
-          if (g >= stages && !mbar_wait(&empty[s], ph ^ 1u, p.status)) {
+          if (g >= stages && !mbar_wait(&empty[s], ph ^ 1u, p.status, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -265,24 +269,26 @@ __global__ void __launch_bounds__(kTCThreads, 1)
       }
       // drain: every issued copy must land before the CTA can exit
       for (int t = max(0, g - stages); t < g; ++t)
-        mbar_wait(&full[t % stages], static_cast<uint32_t>(t / stages) & 1u, p.status);
+        mbar_wait(&full[t % stages], static_cast<uint32_t>(t / stages) & 1u, p.status, p.wait_ns);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t kbase = smem_u32(kst), pbase = smem_u32(pst);
       int g = 0, ii = 0;
-      bool ok = true;
+      // test hook: a wait that runs out before any MMA is issued; every other role then runs out
+      // of its own waits, the producer drains its copies, and the kernel returns SLIM_DEV_TIMEOUT
+      bool ok = !p.stall || mbar_wait(stallbar, 0u, p.status, p.wait_ns);
       while (ok && cur.next(it, s_nb, s_q, s_soff)) {
         const int nt = tiles_of(it);
         // the previous segment's epilogue must have read the accumulator
-        if (ii > 0 && !mbar_wait(accempty, static_cast<uint32_t>(ii - 1) & 1u, p.status)) break;
+        if (ii > 0 && !mbar_wait(accempty, static_cast<uint32_t>(ii - 1) & 1u, p.status, p.wait_ns)) break;
         for (int t = 0; t < nt; ++t, ++g) {
           const int s = g % stages;
           const uint32_t ph = static_cast<uint32_t>(g / stages) & 1u;
           const uint32_t ka = kbase + s * kstage_bytes, pa = pbase + s * pstage_bytes;
           // P of every head in place and the K stage landed
-          if (!mbar_wait<(CL > 1)>(&pfull[s], ph, p.status) || !mbar_wait(&full[s], ph, p.status)) {
+          if (!mbar_wait<(CL > 1)>(&pfull[s], ph, p.status) || !mbar_wait(&full[s], ph, p.status, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -299,7 +305,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
               resc |= (v.x != 1.f) | (v.y != 1.f) | (v.z != 1.f) | (v.w != 1.f);
             }
           }
-          if (resc && !mbar_wait(&corr[s], ph, p.status)) {
+          if (resc && !mbar_wait(&corr[s], ph, p.status, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -319,7 +325,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
           umma_commit(&empty[s]);
           // pempty releases the P stage and its alphas to every writer: the correction warps
           // must have read the alphas first
-          if (!resc && !mbar_wait(&corr[s], ph, p.status)) {
+          if (!resc && !mbar_wait(&corr[s], ph, p.status, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -330,7 +336,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
         ++ii;
       }
       // no MMA may be in flight at teardown: wait for the last commit
-      if (ii > 0) mbar_wait(accfull, static_cast<uint32_t>(ii - 1) & 1u, p.status);
+      if (ii > 0) mbar_wait(accfull, static_cast<uint32_t>(ii - 1) & 1u, p.status, p.wait_ns);
     }
   } else if (warp < 6) {
     // ------------------------------------------------------------ correction + epilogue warpgroup
@@ -349,7 +355,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
       for (int t = 0; t < nt; ++t, ++g) {
         const int s = g % stages;
         const uint32_t ph = static_cast<uint32_t>(g / stages) & 1u;
-        if (!__all_sync(0xffffffffu, mbar_wait<(CL > 1)>(&pfull[s], ph, p.status))) {
+        if (!__all_sync(0xffffffffu, mbar_wait<(CL > 1)>(&pfull[s], ph, p.status, p.wait_ns))) {
           ok = false;
           break;
         }
@@ -358,7 +364,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
           // rescale this quarter's rows once the previous tile's MMAs have finished
           const int sp = (g - 1) % stages;
           const uint32_t php = static_cast<uint32_t>((g - 1) / stages) & 1u;
-          if (!__all_sync(0xffffffffu, mbar_wait(&empty[sp], php, p.status))) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&empty[sp], php, p.status, p.wait_ns))) {
             ok = false;
             break;
           }
@@ -379,7 +385,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
       }
       if (!ok) break;
       // epilogue: accumulator rows -> partial U[slot][head][own columns]
-      if (!__all_sync(0xffffffffu, mbar_wait(accfull, static_cast<uint32_t>(ii) & 1u, p.status))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(accfull, static_cast<uint32_t>(ii) & 1u, p.status, p.wait_ns))) break;
       tc_fence_after();
       float* dst = p.ws_U + (static_cast<size_t>(it.slot) * p.H + max(n, 0)) * p.d + col0 + 512 * hf;
       // four 16-column loads in flight per wait (hcols and my_cols are multiples of 64)
@@ -468,7 +474,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
         const int r_lo = it.row0 + t * TT;
         const int nvalid = min(TT, it.row1 - r_lo);
         const int nloaded = (nvalid + 15) & ~15;
-        if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph, p.status))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph, p.status, p.wait_ns))) {
           ok = false;
           break;
         }
@@ -505,7 +511,7 @@ __global__ void __launch_bounds__(kTCThreads, 1)
 
         // P stage s is free once every CTA's MMAs and copies of tile g - stages finished with
         // it and its correction warps read the alphas (each MMA thread commits after both).
-        if (g >= stages && !__all_sync(0xffffffffu, mbar_wait<(CL > 1)>(&pempty[s], ph ^ 1u, p.status))) {
+        if (g >= stages && !__all_sync(0xffffffffu, mbar_wait<(CL > 1)>(&pempty[s], ph ^ 1u, p.status, p.wait_ns))) {
           ok = false;
           break;
         }
@@ -871,6 +877,8 @@ cudaError_t launch_decode_b_tc(const DecodeArgs& a, const SplitWorkspace& ws, cu
   prm.min_rows = max(16, 8 * a.H);
   prm.tmem_cols = c.tmem_cols;
   prm.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(a.d / a.H));
+  prm.wait_ns = a.wait_ns ? a.wait_ns : kWaitLimitNs;
+  prm.stall = a.stall;
   cudaError_t e = cudaErrorNotSupported;
 #define SLIM_TC_CASE(CL_, TT_, DHB_, HPW_)                           \
   if (c.CL == CL_ && c.TT == TT_ && c.DHB == DHB_ && c.HPW == HPW_) { \

@@ -177,7 +177,8 @@ __global__ void __launch_bounds__(kKVThreads, 1)
       for (int t = 0; t < nt; ++t, ++g) {
         const int s = g % kKVStages;
         const uint32_t ph = static_cast<uint32_t>(g / kKVStages) & 1u;
-        if (!__all_sync(0xffffffffu, mbar_wait(&full[s], ph, p.status))) {
+        // one decision for the four score warps, so their named barriers stay aligned
+        if (!named_barrier_and(1, kKVScoreWarps * 32, __all_sync(0xffffffffu, mbar_wait(&full[s], ph, p.status)))) {
           ok = false;
           break;
         }

@@ -357,6 +357,7 @@ cudaError_t launch_decode_a(const DecodeArgs& a, const SplitWorkspace& ws, cudaS
     if (e != cudaSuccess) return e;
     if (launches) ++*launches;
   }
+  if (decode_a_tc_supported(a.dtype, a.B, a.d, a.H)) return launch_decode_a_tc(a, ws, st, launches);
   e = launch_rows_gemm_any(a.kcache, a.w_kv, ws.vbuf, a.lens, app, a.dtype, a.B, a.d, a.cap, a.status, st,
                            launches);
   if (e != cudaSuccess) return e;

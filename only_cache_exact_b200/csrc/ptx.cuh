@@ -84,18 +84,19 @@ __device__ __forceinline__ uint64_t global_ns() {
 // Bounded wait for phase `parity` of `bar`. try_wait suspends the thread in
 // hardware until the phase completes (or a short hardware limit passes), so
 // the loop polls without sleeping: a sleep would delay every hand-off in the
-// pipeline by its wake-up time. After kWaitLimitNs of the global timer it ORs
-// SLIM_DEV_TIMEOUT into *status and returns false; the caller then leaves its
-// loop and the kernel tears down.
+// pipeline by its wake-up time. After limit_ns of the global timer (by default
+// kWaitLimitNs) it ORs SLIM_DEV_TIMEOUT into *status and returns false; the
+// caller then leaves its loop and the kernel tears down.
 template <bool kCluster = false>
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   const uint32_t a = smem_u32(bar);
   if (kCluster ? mbar_try_wait_cluster(a, parity) : mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = global_ns();
 #pragma unroll 1
   for (uint32_t i = 1;; ++i) {
     if (kCluster ? mbar_try_wait_cluster(a, parity) : mbar_try_wait(a, parity)) return true;
-    if ((i & 63u) == 0u && global_ns() - t0 > kWaitLimitNs) break;
+    if ((i & 63u) == 0u && global_ns() - t0 > limit_ns) break;
   }
   atomicOr(status, SLIM_DEV_TIMEOUT);
   return false;
@@ -110,6 +111,18 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 }
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+// Named barrier that also ANDs a predicate over the participating threads, so a group of warps
+// takes one decision (e.g. to stop after a wait gave up) and stays aligned on its barriers.
+__device__ __forceinline__ bool named_barrier_and(uint32_t id, uint32_t nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
 }
 
 // ------------------------------------------------------------------ TMA

@@ -512,7 +512,7 @@ constexpr int kProjMaxWStages = 16;  // W_KV ring stages at most
 constexpr int kProjDepth = 64;       // U floats in flight per thread
 
 struct ProjSmem {
-  uint32_t w, ub, ubs, wts, soff, part, recv, per, bars, total;
+  uint32_t w, ub, ubs, wts, ls, soff, part, recv, per, bars, total;
 };
 __host__ __device__ inline ProjSmem proj_smem_layout(int DB, int d_h, int nb, int ndb, int ws, int max_items) {
   ProjSmem s;
@@ -522,7 +522,9 @@ __host__ __device__ inline ProjSmem proj_smem_layout(int DB, int d_h, int nb, in
   s.ubs = static_cast<uint32_t>(DB) + 8u;  // row stride of ū (floats): conflict-free fragment loads
   s.ub = o;
   o += up_to(static_cast<uint32_t>(nb), 16u) * s.ubs * 4u;
-  s.wts = o;
+  s.wts = o;  // m of every slot of the launch, then its merge weight
+  o += up_to(static_cast<uint32_t>(max_items), 4u) * 4u;
+  s.ls = o;  // l of every slot of the launch
   o += up_to(static_cast<uint32_t>(max_items), 4u) * 4u;
   s.soff = o;
   o += up_to(static_cast<uint32_t>(nb) + 1u, 4u) * 4u;
@@ -532,16 +534,17 @@ __host__ __device__ inline ProjSmem proj_smem_layout(int DB, int d_h, int nb, in
   s.recv = o;  // products pushed by the cluster's CTAs: [ndb][per]
   o += static_cast<uint32_t>(ndb) * s.per * 4u;
   o = up_to(o, 8u);
-  s.bars = o;
-  o += static_cast<uint32_t>(ws) * 8u;
+  s.bars = o;  // wfull [ws], wempty [ws]
+  o += 2u * static_cast<uint32_t>(ws) * 8u;
   s.total = o + 1024u;  // slack to align the base to 1024 bytes
   return s;
 }
 
 // ū rows of the launch's sequences from their slots (see the kernel's comment); VEC columns per thread.
-template <int VEC>
+template <int VEC, typename Prep>
 __device__ __forceinline__ void proj_merge_rows(const float* ubase, size_t ustride, int nrows, int s_beg,
-                                                const int* s_off, const float* wts, float* ub, int ubs, int tid) {
+                                                const int* s_off, const float* wts, float* ub, int ubs, int tid,
+                                                Prep prep) {
   constexpr int D = kProjDepth / VEC;  // rows in flight
   typedef typename std::conditional<VEC == 4, float4, typename std::conditional<VEC == 2, float2, float>::type>::type
       VT;
@@ -557,6 +560,7 @@ __device__ __forceinline__ void proj_merge_rows(const float* ubase, size_t ustri
     for (int u = 0; u < D; ++u) {
       if (c0 + u < nrows) v[u] = __ldcg(src + static_cast<size_t>(c0 + u) * vstride);
     }
+    if (c0 == 0) prep();  // the merge weights, while the first rows are in flight
 #pragma unroll
     for (int u = 0; u < D; ++u) {
       const int c = c0 + u;
@@ -578,6 +582,8 @@ __device__ __forceinline__ void proj_merge_rows(const float* ubase, size_t ustri
   if (nrows > 0) {
 #pragma unroll
     for (int k = 0; k < VEC; ++k) ub[bl * ubs + VEC * tid + k] = acc[k];
+  } else {
+    prep();
   }
 }
 
@@ -598,10 +604,12 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   uint8_t* wring = sm + L.w;
   float* ub = reinterpret_cast<float*>(sm + L.ub);
   float* wts = reinterpret_cast<float*>(sm + L.wts);
+  float* ls = reinterpret_cast<float*>(sm + L.ls);
   int* s_off = reinterpret_cast<int*>(sm + L.soff);
   float* part = reinterpret_cast<float*>(sm + L.part);
   float* recv = reinterpret_cast<float*>(sm + L.recv);
   uint64_t* wfull = reinterpret_cast<uint64_t*>(sm + L.bars);
+  uint64_t* wempty = wfull + WS;  // every warp is done with the stage
   const int ubs = static_cast<int>(L.ubs), per = static_cast<int>(L.per);
   const int nws = DB / kProjWRows;  // W_KV stages of this block
   constexpr uint32_t kWStageBytes = kProjWRows * DH * 2u;
@@ -620,7 +628,10 @@ __global__ void __launch_bounds__(kProjThreads, 1)
 
   // ---- before the split kernel's results exist
   if (tid == 0) {
-    for (int s = 0; s < WS; ++s) mbar_init(&wfull[s], 1);
+    for (int s = 0; s < WS; ++s) {
+      mbar_init(&wfull[s], 1);
+      mbar_init(&wempty[s], kProjWarps);
+    }
     fence_barrier_init();
     tma_prefetch_desc(&wmap);
     for (int st = 0; st < min(WS, nws); ++st) issue_w(st);
@@ -639,32 +650,41 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   __syncthreads();
   const int s_beg = s_off[0], nrows = s_off[nb] - s_beg;
 
-  // ---- merge weights 2^(m_c - M) / Σ_c' 2^(m_c' - M) l_c', one warp per sequence
-  for (int bl = warp; bl < nb; bl += kProjWarps) {
-    const int lo = s_off[bl], hi = s_off[bl + 1];
-    float M = -INFINITY;
-    for (int c = lo + lane; c < hi; c += 32) M = fmaxf(M, __ldcg(p.m + static_cast<size_t>(c) * p.H + h));
-    M = warp_max(M);
-    float S = 0.f;
-    for (int c = lo + lane; c < hi; c += 32) {
-      const float e = exp2f(__ldcg(p.m + static_cast<size_t>(c) * p.H + h) - M);
-      S = fmaf(e, __ldcg(p.l + static_cast<size_t>(c) * p.H + h), S);
-      wts[c - s_beg] = e;
-    }
-    S = warp_sum(S);
-    const float inv = S > 0.f ? 1.f / S : 0.f;
-    __syncwarp();
-    for (int c = lo + lane; c < hi; c += 32) wts[c - s_beg] *= inv;
+  // ---- m and l of every slot (one load each, all in flight together)
+  for (int c = tid; c < nrows; c += kProjThreads) {
+    wts[c] = __ldcg(p.m + static_cast<size_t>(s_beg + c) * p.H + h);
+    ls[c] = __ldcg(p.l + static_cast<size_t>(s_beg + c) * p.H + h);
   }
-  __syncthreads();
+  // merge weights 2^(m_c - M) / Σ_c' 2^(m_c' - M) l_c', one warp per sequence, from shared memory;
+  // run by proj_merge_rows once its first rows are in flight
+  auto weights = [&]() {
+    __syncthreads();
+    for (int bl = warp; bl < nb; bl += kProjWarps) {
+      const int lo = s_off[bl] - s_beg, hi = s_off[bl + 1] - s_beg;
+      float M = -INFINITY;
+      for (int c = lo + lane; c < hi; c += 32) M = fmaxf(M, wts[c]);
+      M = warp_max(M);
+      float S = 0.f;
+      for (int c = lo + lane; c < hi; c += 32) {
+        const float e = exp2f(wts[c] - M);
+        S = fmaf(e, ls[c], S);
+        ls[c] = e;
+      }
+      S = warp_sum(S);
+      const float inv = S > 0.f ? 1.f / S : 0.f;
+      __syncwarp();
+      for (int c = lo + lane; c < hi; c += 32) wts[c] = ls[c] * inv;
+    }
+    __syncthreads();
+  };
 
   // ---- ū[b, block] = Σ_c w_c U_c[block]
   {
     const float* ubase = p.U + (static_cast<size_t>(s_beg) * p.H + h) * p.d + c0;
     const size_t ustride = static_cast<size_t>(p.H) * p.d;  // floats between slots
-    if (DB == 1024) proj_merge_rows<4>(ubase, ustride, nrows, s_beg, s_off, wts, ub, ubs, tid);
-    else if (DB == 512) proj_merge_rows<2>(ubase, ustride, nrows, s_beg, s_off, wts, ub, ubs, tid);
-    else proj_merge_rows<1>(ubase, ustride, nrows, s_beg, s_off, wts, ub, ubs, tid);
+    if (DB == 1024) proj_merge_rows<4>(ubase, ustride, nrows, s_beg, s_off, wts, ub, ubs, tid, weights);
+    else if (DB == 512) proj_merge_rows<2>(ubase, ustride, nrows, s_beg, s_off, wts, ub, ubs, tid, weights);
+    else proj_merge_rows<1>(ubase, ustride, nrows, s_beg, s_off, wts, ub, ubs, tid, weights);
   }
   __syncthreads();
 
@@ -676,10 +696,15 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     for (int e = 0; e < 4; ++e) acc[i][e] = 0.f;
   const int g = lane >> 2, tq = lane & 3;
   bool ok = true;
-  int w_done = 0;
+  int w_done = 0;  // stages thread 0 has seen released by every warp
   for (int st = 0; st < nws; ++st) {
-    const bool got = mbar_wait(&wfull[st % WS], static_cast<uint32_t>(st / WS) & 1u, p.status);
-    if (got) {
+    const bool got = __all_sync(0xffffffffu, mbar_wait(&wfull[st % WS], static_cast<uint32_t>(st / WS) & 1u,
+                                                        p.status));
+    if (!got) {
+      ok = false;
+      break;
+    }
+    {
       const uint32_t wbase = smem_u32(wring + (st % WS) * kWStageBytes);
 #pragma unroll
       for (int kk = 0; kk < kProjWRows / 16; ++kk) {
@@ -713,11 +738,19 @@ __global__ void __launch_bounds__(kProjThreads, 1)
         }
       }
     }
-    ok = __syncthreads_and(got);  // every warp is done with the stage
-    if (!ok) break;
-    w_done = st + 1;
-    if (tid == 0 && st + WS < nws) issue_w(st + WS);
+    // release the stage; thread 0 refills it once every warp has
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&wempty[st % WS]);
+    if (tid == 0 && st + WS < nws) {
+      if (!mbar_wait(&wempty[st % WS], static_cast<uint32_t>(st / WS) & 1u, p.status)) {
+        ok = false;
+        break;
+      }
+      w_done = st + 1;
+      issue_w(st + WS);
+    }
   }
+  ok = __syncthreads_and(ok);
   if (!ok && tid == 0) {
     // copies still landing in this CTA's shared memory must complete before it exits
     for (int st = w_done; st < w_issued; ++st)

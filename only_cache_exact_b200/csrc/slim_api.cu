@@ -128,20 +128,27 @@ WsLayout ws_layout(int dtype, int B, int d, int H, int64_t cap, int variant) {
   w.max_items = items;
   const bool need_b = variant != SLIM_VARIANT_A;
   const bool need_a = variant != SLIM_VARIANT_B;
-  size_t u_floats = 0;
+  // ordering (a) on tensor cores keeps V in TMEM: one partial of 256 columns (4 heads' m, l) per tile
+  const bool a_tc = need_a && decode_a_tc_supported(dtype, B, d, H);
+  const size_t a_tiles = a_tc ? decode_a_tc_slots(B, d, cap) : 0;
+  size_t u_floats = 0, ml_floats = static_cast<size_t>(items) * H;
   if (need_b) u_floats = std::max(u_floats, static_cast<size_t>(items) * H * d);
-  if (need_a) u_floats = std::max(u_floats, static_cast<size_t>(items) * d);
+  if (need_a && !a_tc) u_floats = std::max(u_floats, static_cast<size_t>(items) * d);
+  if (a_tc) {
+    u_floats = std::max(u_floats, a_tiles * 256);
+    ml_floats = std::max(ml_floats, a_tiles * 4);
+  }
   size_t o = 0;
   w.U = o;
   o += up(u_floats * 4);
   w.m = o;
-  o += up(static_cast<size_t>(items) * H * 4);
+  o += up(ml_floats * 4);
   w.l = o;
-  o += up(static_cast<size_t>(items) * H * 4);
+  o += up(ml_floats * 4);
   w.meta = o;
   o += up(meta_ints(B) * 4);
   w.vbuf = o;
-  if (need_a) o += up(static_cast<size_t>(B) * cap * d * esize(dtype));
+  if (need_a && !a_tc) o += up(static_cast<size_t>(B) * cap * d * esize(dtype));
   w.stage = o;
   o += up(static_cast<size_t>(B) * d * 4) * 2 + up(static_cast<size_t>(B) * d * esize(dtype));
   w.total = o;
@@ -162,6 +169,13 @@ SplitWorkspace carve(void* base, const WsLayout& w) {
 }
 
 thread_local int g_last_launches = 0;
+
+// Test hook of the failure path (slim_debug_stall_next): armed for one call on this thread.
+struct StallHook {
+  uint64_t wait_ns = 0;
+  bool armed = false;
+};
+thread_local StallHook g_stall;
 
 // Measurement aid: event pairs recorded around the split kernel.
 struct TimingRing {
@@ -208,8 +222,6 @@ cudaError_t launch_prefill_simt(const void* X, const void* W, void* kcache, cons
                                 int n, int d, int64_t cap, cudaStream_t st, int* launches);
 cudaError_t launch_prefill_tc(const void* X, const void* W, void* kcache, const int32_t* lens, int B, int n, int d,
                               int64_t cap, int32_t* status, cudaStream_t st, int* launches);
-cudaError_t launch_rows_gemm_tc(const void* A, const void* W, void* Y, const int32_t* lens, int rows_extra, int B,
-                                int d, int64_t cap, int32_t* status, cudaStream_t st, int* launches);
 bool gemm_tc_supported(int d);
 cudaError_t launch_advance_lens(int32_t* lens, int B, int n, int64_t cap, int32_t* status, cudaStream_t st,
                                 int* launches);
@@ -261,6 +273,13 @@ int slim_timing_read(float* ms, int n) {
 }
 
 int slim_last_launch_count(void) { return g_last_launches; }
+
+int slim_debug_stall_next(int64_t wait_ns) {
+  if (wait_ns < 1000 || wait_ns > static_cast<int64_t>(kWaitLimitNs)) return SLIM_EINVAL;
+  g_stall.wait_ns = static_cast<uint64_t>(wait_ns);
+  g_stall.armed = true;
+  return SLIM_OK;
+}
 
 const char* slim_strerror(int code) {
   switch (code) {
@@ -354,6 +373,11 @@ int slim_decode_step(const float* q, const void* k_new, void* Kcache, int32_t* l
   if (v == SLIM_AUTO) v = slim_select_variant(dtype, B, d, H, t_hint > 0 ? t_hint : cap);
 
   DecodeArgs a{q, k_new, Kcache, lens, W_KV, dtype, B, d, H, cap, out, dev_status};
+  if (g_stall.armed && v == SLIM_VARIANT_B) {
+    a.wait_ns = g_stall.wait_ns;
+    a.stall = 1;
+    g_stall.armed = false;
+  }
   SplitWorkspace ws = carve(workspace, wl);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int launches = 0;
@@ -369,6 +393,35 @@ int slim_decode_step(const float* q, const void* k_new, void* Kcache, int32_t* l
     if (!decode_a_supported(dtype, B, d, H)) return SLIM_EUNSUPPORTED;
     e = launch_decode_a(a, ws, st, &launches);
   }
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return e == cudaErrorNotSupported ? SLIM_EUNSUPPORTED : SLIM_ECUDA;
+  }
+  g_last_launches = launches;
+  return SLIM_OK;
+}
+
+size_t slim_prefill_attention_workspace_bytes(int dtype, int B, int d, int H, int64_t cap) {
+  if (!valid_dims(dtype, B, d, H, cap) || !prefill_attn_supported(dtype, d, H)) return 0;
+  return up(static_cast<size_t>(B) * cap * d * esize(dtype));  // V = K·W_KV for the cached rows
+}
+
+int slim_prefill_attention(const void* Q, const void* Kcache, const int32_t* lens, const void* W_KV, int dtype,
+                           int B, int n, int d, int H, int64_t cap, float* out, void* workspace, size_t ws_bytes,
+                           int32_t* dev_status, void* stream) {
+  if (!Q || !Kcache || !lens || !W_KV || !out || !dev_status || n < 1) return SLIM_EINVAL;
+  if (!valid_dims(dtype, B, d, H, cap) || static_cast<int64_t>(n) > cap) return SLIM_EINVAL;
+  if (static_cast<int64_t>(B) * n > (int64_t(1) << 31) - 1) return SLIM_EINVAL;
+  if (!aligned(Q, 16) || !aligned(Kcache, 16) || !aligned(W_KV, 16) || !aligned(out, 16)) return SLIM_EINVAL;
+  if (!prefill_attn_supported(dtype, d, H)) return SLIM_EUNSUPPORTED;
+  const size_t need = slim_prefill_attention_workspace_bytes(dtype, B, d, H, cap);
+  if (!workspace || !aligned(workspace, kAlign) || ws_bytes < need) return SLIM_EWORKSPACE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int launches = 0;
+  // V = K·W_KV for rows 0 .. lens[b]-1 of every sequence, once for all n queries
+  cudaError_t e = launch_rows_gemm_tc(Kcache, W_KV, workspace, lens, 0, B, d, cap, dev_status, st, &launches);
+  if (e == cudaSuccess)
+    e = launch_prefill_attn(Q, Kcache, workspace, lens, B, n, d, H, cap, out, dev_status, st, &launches);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return e == cudaErrorNotSupported ? SLIM_EUNSUPPORTED : SLIM_ECUDA;

@@ -41,6 +41,8 @@ struct DecodeArgs {
   int64_t cap;
   float* out;
   int32_t* status;
+  uint64_t wait_ns = 0;  // 0: kWaitLimitNs
+  int stall = 0;         // test hook (slim_debug_stall_next)
 };
 
 // ---- launchers (return cudaError_t of the launch) ----
@@ -55,7 +57,12 @@ bool decode_b_simt_supported(int B, int d, int H);
 // Merge of variant (b) partials and the W_KV projection; advances lens.
 cudaError_t launch_reduce_b(const DecodeArgs& a, const SplitWorkspace& ws, bool pdl, cudaStream_t st,
                             int* launches);
-// Variant (a): append, V = K·W_KV, split flash-decode over K and V, merge.
+// Variant (a) on tensor cores: V tiles made in TMEM and used there (V never in global memory).
+bool decode_a_tc_supported(int dtype, int B, int d, int H);
+size_t decode_a_tc_slots(int B, int d, int64_t cap);  // tile partials its workspace must hold
+cudaError_t launch_decode_a_tc(const DecodeArgs& a, const SplitWorkspace& ws, cudaStream_t st, int* launches);
+// Variant (a): append, V = K·W_KV, split flash-decode over K and V, merge (the tcgen05 path above
+// where supported).
 cudaError_t launch_decode_a(const DecodeArgs& a, const SplitWorkspace& ws, cudaStream_t st, int* launches);
 bool decode_a_supported(int dtype, int B, int d, int H);
 // Prompt-phase projection K = X·W_K into the cache at lens[b]; then lens += n.
@@ -76,6 +83,15 @@ size_t kv_ws_slots(int B, int d);  // partial slots its workspace needs
 cudaError_t launch_decode_kv(const float* q, const void* k_new, const void* v_new, void* kcache, void* vcache,
                              int32_t* lens, int B, int d, int H, int64_t cap, float* out, float* wsO, float* wsm,
                              float* wsl, int32_t* meta, int32_t* status, cudaStream_t st, int* launches);
+
+// Prompt-phase attention output: causal attention of the n prompt queries over the K-only cache
+// with V = K·W_KV materialised once (ordering (a)).
+bool prefill_attn_supported(int dtype, int d, int H);
+cudaError_t launch_prefill_attn(const void* Q, const void* kcache, const void* vbuf, const int32_t* lens, int B,
+                                int n, int d, int H, int64_t cap, float* out, int32_t* status, cudaStream_t st,
+                                int* launches);
+cudaError_t launch_rows_gemm_tc(const void* A, const void* W, void* Y, const int32_t* lens, int rows_extra, int B,
+                                int d, int64_t cap, int32_t* status, cudaStream_t st, int* launches);
 
 // Tensor map encoding through the driver entry point (no link-time libcuda dependency).
 bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,

@@ -28,7 +28,8 @@ EXPORTS = [
     "slim_prefill_k", "slim_decode_workspace_bytes", "slim_decode_step", "slim_decode_step_host", "slim_tune",
     "slim_tune_record", "slim_select_variant", "slim_tune_clear", "slim_strerror", "slim_last_launch_count",
     "slim_version", "slim_timing_enable", "slim_timing_read", "slim_decode_step_noalloc",
-    "slim_mha_decode_workspace_bytes", "slim_mha_decode_step",
+    "slim_mha_decode_workspace_bytes", "slim_mha_decode_step", "slim_debug_stall_next",
+    "slim_prefill_attention_workspace_bytes", "slim_prefill_attention",
 ]
 
 _vp, _i32, _i64, _sz, _f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
@@ -52,6 +53,10 @@ _SIGS = {
     "slim_decode_step_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i64, _i32, _i64, _vp, _vp,
                                         _vp]),
     "slim_mha_decode_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i64]),
+    "slim_debug_stall_next": (_i32, [_i64]),
+    "slim_prefill_attention_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i64]),
+    "slim_prefill_attention": (_i32, [_vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i64, _vp, _vp, _sz, _vp,
+                                      _vp]),
     "slim_mha_decode_step": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i64, _vp, _vp, _sz, _vp,
                                     _vp]),
 }
@@ -158,6 +163,25 @@ def slim_decode_step_noalloc(q: torch.Tensor, k_new, Kcache: torch.Tensor, lens:
                                          _stream(stream)), "slim_decode_step_noalloc")
 
 
+def slim_prefill_attention_workspace_bytes(dtype: int, B: int, d: int, H: int, cap: int) -> int:
+    return int(_lib.slim_prefill_attention_workspace_bytes(dtype, B, d, H, cap))
+
+
+def slim_prefill_attention(Q: torch.Tensor, Kcache: torch.Tensor, lens: torch.Tensor, W_KV: torch.Tensor, H: int,
+                           out: torch.Tensor, workspace: torch.Tensor, status: torch.Tensor, stream=None) -> None:
+    """Causal attention output of the n prompt queries Q [B][n][d] (bf16) over the K-only cache; out [B][n][d]."""
+    for t, nm in ((Q, "Q"), (Kcache, "Kcache"), (lens, "lens"), (W_KV, "W_KV"), (out, "out"),
+                  (workspace, "workspace"), (status, "status")):
+        _cuda(t, nm)
+    B, n, d = Q.shape
+    cap = Kcache.shape[1]
+    if Kcache.shape != (B, cap, d) or out.shape != (B, n, d) or out.dtype != torch.float32:
+        raise ValueError("shape/dtype mismatch")
+    _check(_lib.slim_prefill_attention(_ptr(Q), _ptr(Kcache), _ptr(lens), _ptr(W_KV), _DT[Q.dtype], B, n, d, H,
+                                       cap, _ptr(out), _ptr(workspace), workspace.numel(), _ptr(status),
+                                       _stream(stream)), "slim_prefill_attention")
+
+
 def slim_mha_decode_workspace_bytes(dtype: int, B: int, d: int, H: int, cap: int) -> int:
     return int(_lib.slim_mha_decode_workspace_bytes(dtype, B, d, H, cap))
 
@@ -237,6 +261,11 @@ def slim_timing_read(n: int) -> list:
     if cnt < 0:
         raise SlimError(cnt, "slim_timing_read")
     return [float(buf[i]) for i in range(cnt)]
+
+
+def slim_debug_stall_next(wait_ns: int) -> None:
+    """Test hook: the next tcgen05 split launch on this thread stalls until its waits (wait_ns) run out."""
+    _check(_lib.slim_debug_stall_next(int(wait_ns)), "slim_debug_stall_next")
 
 
 def raw_lib() -> ctypes.CDLL:
