@@ -92,6 +92,10 @@ def parse():
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling runs)")
     ap.add_argument("--no-extras", action="store_true", help="headline line only (no sub-records, sweep, CPU legs)")
     ap.add_argument("--ref-seconds", type=float, default=20.0, help="CPU time budget of --impl reference")
+    ap.add_argument("--variant", default="auto", choices=["auto", "a", "b"],
+                    help="ordering of the timed steps (auto: the measured table; profiling runs pin one)")
+    ap.add_argument("--from-x", action="store_true",
+                    help="time the step from its input rows (slim_decode_step_x: q and k formed on the device)")
     return ap.parse_args()
 
 
@@ -235,7 +239,8 @@ def cpu_oracle_rate(w, budget_s=12.0):
 class Workload:
     """Device state of one workload: K cache(s) filled by the prompt-phase kernel, W_KV, step inputs."""
 
-    def __init__(self, name, S, dev, rank=0, world=1, max_steps=256, rot=0, mha=False, batch=0):
+    def __init__(self, name, S, dev, rank=0, world=1, max_steps=256, rot=0, mha=False, batch=0, variant=None,
+                 from_x=False):
         import torch
 
         from only_cache_exact_b200 import params, replicas, synth
@@ -291,6 +296,7 @@ class Workload:
         self.fill_s = time.perf_counter() - t
         self.lens_dev0 = lens_dev0
         x_new = np.stack([synth.make_tokens(1, d, 0, gids[b], w["dtype"], part=2)[0] for b in range(B)])
+        self.wts, self.x_new = wts, x_new
         self.q0 = torch.from_numpy(x_new @ wts.W_Q).float().to(dev)
         self.k0 = (synth.to_storage(synth.round_to(x_new @ wts.W_K, w["dtype"]), w["dtype"]).to(dev)
                    if self.append else None)
@@ -309,6 +315,15 @@ class Workload:
                            ws=S.alloc_workspace(self.dt_code, B, d, H, self.cap, S.SLIM_AUTO, device=dev))
             self.sets.append(st_)
         self.t_hint = int(np.max(self.lens0))
+        self.variant = S.SLIM_AUTO if variant is None else variant
+        self.from_x = from_x and not mha
+        if self.from_x:
+            # the step's input rows and the stored W_Q: every timed step forms q (and k) itself
+            self.W_Q = synth.to_storage(synth.round_to(wts.W_Q, w["dtype"]), w["dtype"]).to(dev)
+            self.x = synth.to_storage(x_new, w["dtype"]).to(dev)
+            nws = S.slim_decode_step_x_workspace_bytes(self.dt_code, B, d, H, self.cap, S.SLIM_AUTO)
+            for st_ in self.sets:
+                st_["ws_x"] = torch.empty(nws, dtype=torch.uint8, device=dev)
         self.stream = torch.cuda.Stream(device=dev)
         self.flush_buf = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev) if self.flush else None
         torch.cuda.synchronize()
@@ -320,8 +335,13 @@ class Workload:
             S.slim_mha_decode_step(s["q"], s["k"], s["v"], s["K"], s["V"], s["lens"], self.H, s["out"], s["ws"],
                                    self.status)
             return
+        v = self.variant if variant is None else variant
+        if self.from_x:
+            S.slim_decode_step_x(self.x, self.W_Q, self.W_K if self.append else None, s["K"], s["lens"], s["W_KV"],
+                                 self.H, s["out"], s["ws_x"], self.status, variant=v, t_hint=self.t_hint)
+            return
         S.slim_decode_step(s["q"], s["k"], s["K"], s["lens"], s["W_KV"], self.H, s["out"], s["ws"], self.status,
-                           variant=S.SLIM_AUTO if variant is None else variant, t_hint=self.t_hint)
+                           variant=v, t_hint=self.t_hint)
 
     def reset_lengths(self):
         import torch
@@ -464,7 +484,8 @@ class Workload:
         ms = replicas.max_over_ranks(ms, pg, self.dev)
         st = int(self.status.item())
         ms_step = ms / K_steps
-        chosen = S.slim_select_variant(self.dt_code, self.B, self.d, self.H, self.t_hint)
+        chosen = (self.variant if self.variant != S.SLIM_AUTO
+                  else S.slim_select_variant(self.dt_code, self.B, self.d, self.H, self.t_hint))
         launches = S.slim_last_launch_count()
         n_live = min(max(K_steps, 8), 64)
         split_ms = None if self.mha else self.split_kernel_ms(n_live)
@@ -477,6 +498,57 @@ class Workload:
                  peak_src=peak_src)
         r["e2e_ms"] = self.e2e_ms(max(8, min(K_steps, 200)), pg) if e2e and not self.mha else None
         return r
+
+    def front_end(self, n=20):
+        """The step started from its input rows (slim_decode_step_x: q = x·W_Q and, with append,
+        k = x·W_K formed on the device) against the step handed q and k (slim_decode_step): n steps
+        of each behind a spin kernel, from the same starting lengths. None for workloads timed with
+        an L2 flush per step."""
+        import torch
+
+        from only_cache_exact_b200 import synth
+        if self.flush or self.mha:
+            return None
+        S, dt = self.S, self.w["dtype"]
+        W_Q = synth.to_storage(synth.round_to(self.wts.W_Q, dt), dt).to(self.dev)
+        W_K = self.W_K if self.append else None
+        x = synth.to_storage(self.x_new, dt).to(self.dev)
+        nws = S.slim_decode_step_x_workspace_bytes(self.dt_code, self.B, self.d, self.H, self.cap, S.SLIM_AUTO)
+        ws_x = [torch.empty(nws, dtype=torch.uint8, device=self.dev) for _ in range(self.rot)]
+
+        def plain(i):
+            s = self.sets[i % self.rot]
+            S.slim_decode_step(s["q"], s["k"], s["K"], s["lens"], s["W_KV"], self.H, s["out"], s["ws"], self.status,
+                               variant=S.SLIM_AUTO, t_hint=self.t_hint)
+
+        def from_x(i):
+            s = self.sets[i % self.rot]
+            S.slim_decode_step_x(x, W_Q, W_K, s["K"], s["lens"], s["W_KV"], self.H, s["out"], ws_x[i % self.rot],
+                                 self.status, variant=S.SLIM_AUTO, t_hint=self.t_hint)
+
+        def timed(fn):
+            self.reset_lengths()
+            for i in range(3):
+                fn(i)
+            self.stream.synchronize()
+            self.reset_lengths()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(self.stream):
+                torch.cuda._sleep(int(50e6))
+                e0.record(self.stream)
+                for i in range(n):
+                    fn(i)
+                e1.record(self.stream)
+            e1.synchronize()
+            return e0.elapsed_time(e1) / n
+
+        ms_q = timed(plain)
+        ms_x = timed(from_x)
+        launches = S.slim_last_launch_count()
+        del ws_x
+        return {"steps": n, "ms_per_step_from_q": ms_q, "ms_per_step_from_x": ms_x,
+                "front_end_ms": ms_x - ms_q, "launches_per_step_from_x": launches,
+                "projections": "q and k" if self.append else "q only (cross-attention)"}
 
     def l2_note(self):
         if self.flush:
@@ -513,6 +585,7 @@ def sub_record(name, S, dev, cpu_budget):
     w = WORKLOADS[name]
     wl = Workload(name, S, dev, max_steps=max(w["steps"], 64) + 8)
     r = wl.measure(w["steps"], 3)
+    front = wl.front_end()
     rate, threads, n, T = cpu_oracle_rate(w, budget_s=cpu_budget)
     rec = {"workload": w["desc"], "steps": w["steps"], "warmup": 3, "ms_per_step": r["ms_step"],
            "steps_per_s": 1e3 / r["ms_step"], "tokens_per_s": 1e3 / r["ms_step"] * w["B"],
@@ -521,7 +594,7 @@ def sub_record(name, S, dev, cpu_budget):
            "ordering": {1: "a", 2: "b"}.get(r["chosen"], "?"), "launches_per_step": r["launches"],
            "roofline": roofline_record(name, r),
            "e2e": {"value": 1e3 / r["e2e_ms"], "unit": "steps/s"} if r["e2e_ms"] else None,
-           "l2": wl.l2_note(), "footprint": wl.footprint(), "status": r["status"],
+           "l2": wl.l2_note(), "footprint": wl.footprint(), "status": r["status"], "front_end": front,
            "cpu_baseline": {"value": rate, "unit": "steps/s", "cores": threads, "kind": "oracle",
                             "sample": f"{n} single-sequence float64 oracle steps at T={T}, scaled to the batch"}}
     del wl
@@ -701,6 +774,47 @@ def run_variant_a(S, dev):
             "frac_of_bf16_peak": flops / (ms_a * 1e-3) / 1e12 / tc_peak}
 
 
+def run_front_kernel(S, dev):
+    """The front-end kernel alone (slim_project_qk) on the batch shapes of the decode workloads: it
+    reads W_Q (and W_K) once, so its roofline is HBM at 2·d² bytes per projection plus the rows.
+    Each call is timed alone after a 256 MB write (the weights would otherwise sit in L2)."""
+    import torch
+    hbm_peak, _, _ = peaks()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(11)
+    out = {}
+    for d, B, with_k in ((1024, 8, True), (4096, 16, True), (1280, 64, False), (4096, 1, True)):
+        x = torch.randn(B, d, generator=g, device=dev).to(torch.bfloat16)
+        W_Q = (torch.randn(d, d, generator=g, device=dev) / d ** 0.5).to(torch.bfloat16)
+        W_K = (torch.randn(d, d, generator=g, device=dev) / d ** 0.5).to(torch.bfloat16) if with_k else None
+        q = torch.empty(B, d, dtype=torch.float32, device=dev)
+        k = torch.empty(B, d, dtype=torch.bfloat16, device=dev) if with_k else None
+        for _ in range(3):
+            S.slim_project_qk(x, W_Q, W_K, q, k, status)
+        torch.cuda.synchronize()
+        reps, tot = 10, 0.0
+        for i in range(reps):
+            flush.fill_(i & 0xFF)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            S.slim_project_qk(x, W_Q, W_K, q, k, status)
+            e1.record()
+            e1.synchronize()
+            tot += e0.elapsed_time(e1)
+        ms = tot / reps
+        nproj = 2 if with_k else 1
+        nbytes = nproj * d * d * 2 + B * d * 2 + B * d * 4 + (B * d * 2 if with_k else 0)
+        out[f"d{d}_b{B}_{'qk' if with_k else 'q'}"] = {
+            "ms": ms, "bytes": nbytes, "hbm_gbs": nbytes / (ms * 1e-3) / 1e9,
+            "frac": nbytes / (ms * 1e-3) / 1e9 / hbm_peak, "status": int(status.item())}
+        del x, W_Q, W_K, q, k
+    del flush
+    torch.cuda.empty_cache()
+    return out
+
+
 # ------------------------------------------------------------------------------------------ main
 def main():
     args = parse()
@@ -733,12 +847,17 @@ def main():
     from only_cache_exact_b200 import replicas, slim as S
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    variant = {"auto": S.SLIM_AUTO, "a": S.SLIM_VARIANT_A, "b": S.SLIM_VARIANT_B}[args.variant]
     wl = Workload(args.workload, S, dev, rank, world, max_steps=max(args.steps, args.warmup, 64) + 8,
-                  rot=args.rot, batch=args.batch)
+                  rot=args.rot, batch=args.batch, variant=variant, from_x=args.from_x)
     if args.batch:  # a reduced batch for profiling captures; the line says so
         w = wl.w
         workload_cfg["B"] = w["B"]
         workload_cfg["workload"] += f" (batch reduced to {w['B']})"
+    if args.variant != "auto":
+        workload_cfg["ordering"] = args.variant
+    if args.from_x:
+        workload_cfg["from_input_rows"] = True
     sampler = ClockSampler(local)
     r = wl.measure(args.steps, args.warmup, pg, sampler)
     cfg = dict(workload_cfg)
@@ -748,6 +867,7 @@ def main():
     h2d = int(w["B"] * w["d"] * 4 + (w["B"] * w["d"] * wl.esz if wl.append else 0))
     d2h = int(w["B"] * w["d"] * 4)
     footprint = wl.footprint()
+    front = wl.front_end() if not args.no_extras else None
     del wl
     torch.cuda.empty_cache()
 
@@ -761,6 +881,7 @@ def main():
         extras["sweep"], extras["prefill"] = run_sweep(S, dev)
         extras["prefill_d1024"] = run_prefill_d1024(S, dev)
         extras["variant_a"] = run_variant_a(S, dev)
+        extras["front_end_kernel"] = run_front_kernel(S, dev)
 
     if rank != 0:
         if pg:
@@ -789,6 +910,7 @@ def main():
             "launches_per_step": r["launches"],
             "clocks": sampler.summary(),
             "footprint": footprint,
+            "front_end": front,
             "status": r["status"]}
     line.update(extras)
     print(json.dumps(line))

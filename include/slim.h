@@ -137,6 +137,44 @@ int slim_decode_step_host(const float* q_host, const void* k_new_host, void* Kca
                           float* out_host, void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream);
 
 /*
+ * slim_project_qk — the step's front end: q = x·W_Q and, for self-attention,
+ * k = x·W_K for the B input rows of one generation step. Source: section
+ * "K-Cache is All You Need", generation phase (the step computes the query of
+ * the new token, scores it against the cached K, and appends the new token's
+ * key k to the cache; row vectors, as in K = X·W_K).
+ *
+ *   x       [B][d] in `dtype`      this step's input rows (device, read)
+ *   W_Q     [d][d] in `dtype`      (device, read)
+ *   W_K     [d][d] in `dtype`, or NULL: q only (a cross-attention step)
+ *   dtype   SLIM_BF16: tcgen05 tensor cores where d % 128 == 0 (fp32
+ *           accumulation in an order the hardware fixes; k rounded once to
+ *           bf16, round-to-nearest-even), CUDA cores otherwise;
+ *           SLIM_F32: one fp32 accumulator per output, reduction index
+ *           ascending, one fused multiply-add per step (bitwise reproducible)
+ *   q_out   float[B][d]            (device, written)
+ *   k_out   [B][d] in `dtype`      (device, written); NULL exactly when W_K is
+ *   dev_status  device int32 (SLIM_DEV_TIMEOUT only)
+ * All pointers 16-byte aligned; SLIM_BF16 needs d % 8 == 0, SLIM_F32 d % 4 == 0.
+ */
+int slim_project_qk(const void* x, const void* W_Q, const void* W_K, int dtype, int B, int d, float* q_out,
+                    void* k_out, int32_t* dev_status, void* stream);
+
+/*
+ * slim_decode_step_x — slim_decode_step that starts from the step's input
+ * rows: the front end above computes q = x·W_Q and (W_K != NULL) k = x·W_K
+ * into the workspace, and the step then attends exactly as slim_decode_step
+ * does with those q and k_new (W_K == NULL: cross-attention, no append). Its
+ * result equals, bit for bit, slim_project_qk followed by slim_decode_step on
+ * the same arguments. The workspace must hold
+ * slim_decode_step_x_workspace_bytes(...) bytes (the step's scratch plus q and
+ * k); other arguments as for slim_decode_step and slim_project_qk.
+ */
+size_t slim_decode_step_x_workspace_bytes(int dtype, int B, int d, int H, int64_t cap, int variant);
+int slim_decode_step_x(const void* x, const void* W_Q, const void* W_K, void* Kcache, int32_t* lens,
+                       const void* W_KV, int dtype, int B, int d, int H, int64_t cap, int variant, int64_t t_hint,
+                       float* out, void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/*
  * slim_decode_step_noalloc — slim_decode_step without a caller workspace, for
  * callers that cannot allocate device memory: a plug-in whose host runtime
  * owns all device memory under a plan fixed at start-up and passes it only

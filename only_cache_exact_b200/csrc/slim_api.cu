@@ -401,6 +401,56 @@ int slim_decode_step(const float* q, const void* k_new, void* Kcache, int32_t* l
   return SLIM_OK;
 }
 
+int slim_project_qk(const void* x, const void* W_Q, const void* W_K, int dtype, int B, int d, float* q_out,
+                    void* k_out, int32_t* dev_status, void* stream) {
+  if (!x || !W_Q || !q_out || !dev_status || (!W_K != !k_out)) return SLIM_EINVAL;
+  if (!valid_dims(dtype, B, d, 1, 1)) return SLIM_EINVAL;
+  if (!aligned(x, 16) || !aligned(W_Q, 16) || (W_K && !aligned(W_K, 16)) || !aligned(q_out, 16) ||
+      (k_out && !aligned(k_out, 16)))
+    return SLIM_EINVAL;
+  if ((static_cast<size_t>(d) * esize(dtype)) % 16 != 0) return SLIM_EUNSUPPORTED;
+  int launches = 0;
+  const cudaError_t e = launch_front(x, W_Q, W_K, q_out, k_out, dtype, B, d, dev_status,
+                                     static_cast<cudaStream_t>(stream), &launches);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return SLIM_ECUDA;
+  }
+  g_last_launches = launches;
+  return SLIM_OK;
+}
+
+size_t slim_decode_step_x_workspace_bytes(int dtype, int B, int d, int H, int64_t cap, int variant) {
+  const size_t step = slim_decode_workspace_bytes(dtype, B, d, H, cap, variant);
+  if (step == 0) return 0;
+  return step + up(static_cast<size_t>(B) * d * 4) + up(static_cast<size_t>(B) * d * esize(dtype));
+}
+
+int slim_decode_step_x(const void* x, const void* W_Q, const void* W_K, void* Kcache, int32_t* lens,
+                       const void* W_KV, int dtype, int B, int d, int H, int64_t cap, int variant, int64_t t_hint,
+                       float* out, void* workspace, size_t ws_bytes, int32_t* dev_status, void* stream) {
+  // the step's own checks first, so that a rejected call launches nothing
+  if (!x || !W_Q || !Kcache || !lens || !W_KV || !out || !dev_status) return SLIM_EINVAL;
+  if (!valid_dims(dtype, B, d, H, cap) || variant < SLIM_AUTO || variant > SLIM_VARIANT_B) return SLIM_EINVAL;
+  if (!aligned(x, 16) || !aligned(W_Q, 16) || (W_K && !aligned(W_K, 16)) || !aligned(Kcache, 16) ||
+      !aligned(W_KV, 16))
+    return SLIM_EINVAL;
+  if ((static_cast<size_t>(d) * esize(dtype)) % 16 != 0) return SLIM_EUNSUPPORTED;
+  if (!workspace || !aligned(workspace, kAlign)) return SLIM_EWORKSPACE;
+  const size_t step = ws_layout(dtype, B, d, H, cap, variant).total;
+  if (ws_bytes < slim_decode_step_x_workspace_bytes(dtype, B, d, H, cap, variant)) return SLIM_EWORKSPACE;
+  char* w = static_cast<char*>(workspace);
+  float* q = reinterpret_cast<float*>(w + step);
+  void* k = W_K ? w + step + up(static_cast<size_t>(B) * d * 4) : nullptr;
+  int r = slim_project_qk(x, W_Q, W_K, dtype, B, d, q, k, dev_status, stream);
+  if (r != SLIM_OK) return r;
+  const int front_launches = g_last_launches;
+  r = slim_decode_step(q, k, Kcache, lens, W_KV, dtype, B, d, H, cap, variant, t_hint, out, workspace, step,
+                       dev_status, stream);
+  if (r == SLIM_OK) g_last_launches += front_launches;
+  return r;
+}
+
 size_t slim_prefill_attention_workspace_bytes(int dtype, int B, int d, int H, int64_t cap) {
   if (!valid_dims(dtype, B, d, H, cap) || !prefill_attn_supported(dtype, d, H)) return 0;
   return up(static_cast<size_t>(B) * cap * d * esize(dtype));  // V = K·W_KV for the cached rows

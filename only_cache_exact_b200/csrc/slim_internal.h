@@ -93,6 +93,12 @@ cudaError_t launch_prefill_attn(const void* Q, const void* kcache, const void* v
 cudaError_t launch_rows_gemm_tc(const void* A, const void* W, void* Y, const int32_t* lens, int rows_extra, int B,
                                 int d, int64_t cap, int32_t* status, cudaStream_t st, int* launches);
 
+// Step front end: q = x·W_Q (fp32) and, with W_K, k = x·W_K (cache dtype) for B input rows.
+bool front_tc_supported(int dtype, int d);
+int front_tc_split(int d, bool with_k);  // cluster size of the tcgen05 front end
+cudaError_t launch_front(const void* x, const void* W_Q, const void* W_K, float* q, void* k, int dtype, int B, int d,
+                         int32_t* status, cudaStream_t st, int* launches);
+
 // Tensor map encoding through the driver entry point (no link-time libcuda dependency).
 bool encode_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer, uint64_t row_bytes,
                          uint32_t box_inner, uint32_t box_outer, bool swizzle128);

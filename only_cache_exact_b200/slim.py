@@ -29,7 +29,8 @@ EXPORTS = [
     "slim_tune_record", "slim_select_variant", "slim_tune_clear", "slim_strerror", "slim_last_launch_count",
     "slim_version", "slim_timing_enable", "slim_timing_read", "slim_decode_step_noalloc",
     "slim_mha_decode_workspace_bytes", "slim_mha_decode_step", "slim_debug_stall_next",
-    "slim_prefill_attention_workspace_bytes", "slim_prefill_attention",
+    "slim_prefill_attention_workspace_bytes", "slim_prefill_attention", "slim_project_qk",
+    "slim_decode_step_x_workspace_bytes", "slim_decode_step_x",
 ]
 
 _vp, _i32, _i64, _sz, _f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
@@ -59,6 +60,10 @@ _SIGS = {
                                       _vp]),
     "slim_mha_decode_step": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i64, _vp, _vp, _sz, _vp,
                                     _vp]),
+    "slim_project_qk": (_i32, [_vp, _vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp]),
+    "slim_decode_step_x_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i64, _i32]),
+    "slim_decode_step_x": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i64, _i32, _i64, _vp, _vp,
+                                  _sz, _vp, _vp]),
 }
 SLIM_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 for _name, (_res, _args) in _SIGS.items():
@@ -149,6 +154,51 @@ def slim_decode_step(q: torch.Tensor, k_new, Kcache: torch.Tensor, lens: torch.T
     _check(_lib.slim_decode_step(_ptr(q), _ptr(k_new), _ptr(Kcache), _ptr(lens), _ptr(W_KV), _DT[Kcache.dtype],
                                  B, d, H, cap, variant, t_hint, _ptr(out), _ptr(workspace), workspace.numel(),
                                  _ptr(status), _stream(stream)), "slim_decode_step")
+
+
+def slim_project_qk(x: torch.Tensor, W_Q: torch.Tensor, W_K, q_out: torch.Tensor, k_out, status: torch.Tensor,
+                    stream=None) -> None:
+    """Step front end: q_out = x·W_Q (fp32 [B][d]) and, with W_K, k_out = x·W_K ([B][d] in x's dtype)."""
+    for t, nm in ((x, "x"), (W_Q, "W_Q"), (q_out, "q_out"), (status, "status")):
+        _cuda(t, nm)
+    B, d = x.shape
+    if W_Q.shape != (d, d) or W_Q.dtype != x.dtype or q_out.shape != (B, d) or q_out.dtype != torch.float32:
+        raise ValueError("shape/dtype mismatch")
+    if (W_K is None) != (k_out is None):
+        raise ValueError("W_K and k_out go together")
+    if W_K is not None:
+        _cuda(W_K, "W_K")
+        _cuda(k_out, "k_out")
+        if W_K.shape != (d, d) or W_K.dtype != x.dtype or k_out.shape != (B, d) or k_out.dtype != x.dtype:
+            raise ValueError("shape/dtype mismatch")
+    _check(_lib.slim_project_qk(_ptr(x), _ptr(W_Q), _ptr(W_K), _DT[x.dtype], B, d, _ptr(q_out), _ptr(k_out),
+                                _ptr(status), _stream(stream)), "slim_project_qk")
+
+
+def slim_decode_step_x_workspace_bytes(dtype: int, B: int, d: int, H: int, cap: int, variant: int = SLIM_AUTO) -> int:
+    return int(_lib.slim_decode_step_x_workspace_bytes(dtype, B, d, H, cap, variant))
+
+
+def slim_decode_step_x(x: torch.Tensor, W_Q: torch.Tensor, W_K, Kcache: torch.Tensor, lens: torch.Tensor,
+                       W_KV: torch.Tensor, H: int, out: torch.Tensor, workspace: torch.Tensor, status: torch.Tensor,
+                       variant: int = SLIM_AUTO, t_hint: int = 0, stream=None) -> None:
+    """One generation step from the input rows x [B][d] (cache dtype): q = x·W_Q, k = x·W_K (W_K None: no
+    append), then the step as slim_decode_step."""
+    for t, nm in ((x, "x"), (W_Q, "W_Q"), (Kcache, "Kcache"), (lens, "lens"), (W_KV, "W_KV"), (out, "out"),
+                  (workspace, "workspace"), (status, "status")):
+        _cuda(t, nm)
+    B, cap, d = Kcache.shape
+    if x.shape != (B, d) or x.dtype != Kcache.dtype or W_Q.shape != (d, d) or W_Q.dtype != x.dtype:
+        raise ValueError("x/W_Q must be [B][d]/[d][d] in the cache dtype")
+    if W_K is not None:
+        _cuda(W_K, "W_K")
+        if W_K.shape != (d, d) or W_K.dtype != x.dtype:
+            raise ValueError("W_K must be [d][d] in the cache dtype")
+    if out.shape != (B, d) or out.dtype != torch.float32:
+        raise ValueError("out must be float32 [B][d]")
+    _check(_lib.slim_decode_step_x(_ptr(x), _ptr(W_Q), _ptr(W_K), _ptr(Kcache), _ptr(lens), _ptr(W_KV),
+                                   _DT[Kcache.dtype], B, d, H, cap, variant, t_hint, _ptr(out), _ptr(workspace),
+                                   workspace.numel(), _ptr(status), _stream(stream)), "slim_decode_step_x")
 
 
 def slim_decode_step_noalloc(q: torch.Tensor, k_new, Kcache: torch.Tensor, lens: torch.Tensor, W_KV: torch.Tensor,

@@ -97,6 +97,46 @@ def test_prefill_rejects_bad_arguments(S):
     assert L.slim_prefill_k(f, f, f, f, 3, 1, 8, 256, 64, f, None) == S.SLIM_EINVAL
 
 
+def test_front_end_rejects_bad_arguments_without_launch(S):
+    """slim_project_qk and slim_decode_step_x check every argument before launching anything."""
+    L = S.raw_lib()
+    f = ctypes.c_void_p(1 << 20)
+    odd = ctypes.c_void_p((1 << 20) + 8)
+
+    def proj(x=f, wq=f, wk=f, dt=S.SLIM_BF16, B=8, d=1024, q=f, k=f, st=f):
+        return L.slim_project_qk(x, wq, wk, dt, B, d, q, k, st, None)
+
+    assert proj(x=None) == S.SLIM_EINVAL
+    assert proj(wq=None) == S.SLIM_EINVAL
+    assert proj(q=None) == S.SLIM_EINVAL
+    assert proj(st=None) == S.SLIM_EINVAL
+    assert proj(k=None) == S.SLIM_EINVAL  # W_K without k_out
+    assert proj(wk=None) == S.SLIM_EINVAL  # k_out without W_K
+    assert proj(dt=4) == S.SLIM_EINVAL
+    assert proj(B=0) == S.SLIM_EINVAL
+    assert proj(x=odd) == S.SLIM_EINVAL
+    assert proj(d=1020) == S.SLIM_EUNSUPPORTED  # a bf16 row of 2040 bytes is not a 16-byte multiple
+
+    def step(x=f, wq=f, wk=f, K=f, lens=f, w=f, d=1024, H=16, v=0, out=f, ws=f, wsb=1 << 40, st=f):
+        return L.slim_decode_step_x(x, wq, wk, K, lens, w, S.SLIM_BF16, 8, d, H, 4160, v, 0, out, ws, wsb, st, None)
+
+    assert step(x=None) == S.SLIM_EINVAL
+    assert step(wq=None) == S.SLIM_EINVAL
+    assert step(K=None) == S.SLIM_EINVAL
+    assert step(w=None) == S.SLIM_EINVAL
+    assert step(out=None) == S.SLIM_EINVAL
+    assert step(d=1000) == S.SLIM_EINVAL
+    assert step(v=5) == S.SLIM_EINVAL
+    assert step(wk=odd) == S.SLIM_EINVAL
+    assert step(ws=None) == S.SLIM_EWORKSPACE
+    need = S.slim_decode_step_x_workspace_bytes(S.SLIM_BF16, 8, 1024, 16, 4160, S.SLIM_AUTO)
+    assert step(wsb=need - 1) == S.SLIM_EWORKSPACE
+    # the step's scratch plus q (fp32) and k (cache dtype), each rounded up to 256 bytes
+    base = S.slim_decode_workspace_bytes(S.SLIM_BF16, 8, 1024, 16, 4160, S.SLIM_AUTO)
+    assert need == base + 8 * 1024 * 4 + 8 * 1024 * 2
+    assert S.slim_decode_step_x_workspace_bytes(S.SLIM_BF16, 8, 1000, 16, 4160, 0) == 0
+
+
 def test_host_entry_rejects_bad_arguments_before_any_copy(S):
     """Every argument check precedes the host-to-device copies: with fake device pointers that
     would fault if a copy were enqueued, a bad call returns its error code and does nothing."""
