@@ -478,20 +478,25 @@ __global__ void __launch_bounds__(kLeanThreads, 1)
 // ---------------------------------------------------------------------------- projection merge
 // bf16 W_KV, d_h = 64 DHB (DHB = 1 or 2), up to 16 MT sequences per launch. Grid (H, NDB),
 // clusters of NDB CTAs along y; CTA (h, r) owns head h and the rows [r·DB, (r+1)·DB) of W_KV,
-// DB = 256 VEC (VEC = 1, 2 or 4).
-//   * Before the split kernel's results are awaited: barriers, zeroed ū, and the first
-//     `ws` tiles of W_KV[block rows, head-h columns] (64 rows x 64 columns per TMA box,
+// DB = 256, 512 or 1024.
+//   * Before the split kernel's results are awaited: barriers, TMEM, a zeroed ū operand, and the
+//     first `ws` tiles of W_KV[block rows, head-h columns] (64 rows x 64 columns per TMA box,
 //     128-byte swizzle) requested into a ring of `ws` stages.
-//   * The slot range of the launch's sequences and, one warp per sequence, the merge weights
-//     from the slots' m and l.
-//   * ū[b, block] = Σ_c w_c U_c[block]: thread t owns the VEC columns VEC t ..; it loads its
-//     part of kProjDepth / VEC slots' rows at once (plain loads, all in flight together, no
-//     barrier) and adds them in slot order, so a sequence's sum is finished when its last slot
-//     has been added and the order of the additions is fixed.
-//   * o_r[b, :] = ū[b, block] · W_KV[block, h-cols] on mma.sync m16n8k16 (ū as a bf16 high and
-//     low part, fp32 accumulation), the W_KV tiles streamed through the ring.
-//   * The NDB products of an output element are pushed to one owner CTA and added there in a
-//     fixed order, so the result does not depend on timing.
+//   * The slot range of the launch's sequences, every slot's m and l and its sequence.
+//   * ū[b, block] = Σ_c w_c U_c[block]: thread t owns DB/256 columns and keeps 64 floats of
+//     partial rows in flight (plain loads, no barrier: the rows were just written by the split
+//     kernel and are read once, so what matters is having many requests outstanding); the merge
+//     weights w_c = 2^(m_c - M) / Σ 2^(m_c' - M) l_c' are formed, one warp per sequence, while the
+//     first rows are in flight. Rows are added in slot order (a fixed order: deterministic); when a
+//     sequence's last row has been added its sum is written as the bf16 high and low parts of the
+//     MMA operand (K-major, 128-byte swizzle), so that the projection keeps fp32 accuracy on bf16
+//     tensor ops.
+//   * o_r = W_KV[block, h-cols]^T · ū^T on tcgen05 (M = d_h, N = 16 MT sequences, K = 16 rows of
+//     the block per MMA; W_KV read in place from the ring as the MN-major operand, the high and
+//     low parts accumulated into one fp32 TMEM accumulator), a ring stage refilled three stages
+//     after its MMAs were issued.
+//   * The NDB products of an output element are pushed to one owner CTA through distributed
+//     shared memory and added there in a fixed order, so the result does not depend on timing.
 struct MergeProjParams {
   const float* U;
   const float* m;
@@ -509,51 +514,64 @@ constexpr int kProjThreads = 256;
 constexpr int kProjWarps = kProjThreads / 32;
 constexpr int kProjWRows = 64;       // W_KV rows per ring stage
 constexpr int kProjMaxWStages = 16;  // W_KV ring stages at most
-constexpr int kProjDepth = 64;       // U floats in flight per thread
+constexpr int kProjDepth = 64;       // partial-row floats in flight per thread
 
 struct ProjSmem {
-  uint32_t w, ub, ubs, wts, ls, soff, part, recv, per, bars, total;
+  uint32_t w, ub, part, recv, per, wts, ls, rseq, soff, bars, slot, total;
 };
+// BP = 16 MT sequences (the MMA's N)
 __host__ __device__ inline ProjSmem proj_smem_layout(int DB, int d_h, int nb, int ndb, int ws, int max_items) {
   ProjSmem s;
+  const uint32_t BP = up_to(static_cast<uint32_t>(nb), 16u);
   uint32_t o = 0;
-  s.w = o;  // [ws][d_h / 64 boxes][64 rows][128 bytes], each stage a multiple of 1024 bytes
+  s.w = o;  // [ws][d_h / 64 boxes][64 rows][128 bytes]
   o += static_cast<uint32_t>(ws) * kProjWRows * d_h * 2u;
-  s.ubs = static_cast<uint32_t>(DB) + 8u;  // row stride of ū (floats): conflict-free fragment loads
-  s.ub = o;
-  o += up_to(static_cast<uint32_t>(nb), 16u) * s.ubs * 4u;
+  s.ub = o;  // ū in bf16, high then low part: [2][DB / 64 chunks][BP rows][128 bytes], swizzled
+  o += 2u * static_cast<uint32_t>(DB) * BP * 2u;
+  s.part = o;  // this CTA's products [nb][d_h]
+  o += up_to(static_cast<uint32_t>(nb) * d_h * 4u, 16u);
+  s.per = (static_cast<uint32_t>(nb) * d_h + ndb - 1u) / ndb;
+  s.recv = o;  // products pushed by the cluster's CTAs: [ndb][per]
+  o += up_to(static_cast<uint32_t>(ndb) * s.per * 4u, 16u);
   s.wts = o;  // m of every slot of the launch, then its merge weight
   o += up_to(static_cast<uint32_t>(max_items), 4u) * 4u;
   s.ls = o;  // l of every slot of the launch
   o += up_to(static_cast<uint32_t>(max_items), 4u) * 4u;
+  s.rseq = o;  // sequence (within the launch) of every slot
+  o += up_to(static_cast<uint32_t>(max_items), 4u) * 4u;
   s.soff = o;
   o += up_to(static_cast<uint32_t>(nb) + 1u, 4u) * 4u;
-  s.part = o;  // this CTA's product [nb][d_h]
-  o += static_cast<uint32_t>(nb) * d_h * 4u;
-  s.per = (static_cast<uint32_t>(nb) * d_h + ndb - 1u) / ndb;
-  s.recv = o;  // products pushed by the cluster's CTAs: [ndb][per]
-  o += static_cast<uint32_t>(ndb) * s.per * 4u;
   o = up_to(o, 8u);
-  s.bars = o;  // wfull [ws], wempty [ws]
-  o += 2u * static_cast<uint32_t>(ws) * 8u;
+  s.bars = o;  // wfull [ws], wempty [ws], accbar
+  o += (2u * static_cast<uint32_t>(ws) + 1u) * 8u;
+  s.slot = o;  // TMEM address, failure flag
+  o += 16u;
   s.total = o + 1024u;  // slack to align the base to 1024 bytes
   return s;
 }
 
-// ū rows of the launch's sequences from their slots (see the kernel's comment); VEC columns per thread.
-template <int VEC, typename Prep>
-__device__ __forceinline__ void proj_merge_rows(const float* ubase, size_t ustride, int nrows, int s_beg,
-                                                const int* s_off, const float* wts, float* ub, int ubs, int tid,
-                                                Prep prep) {
-  constexpr int D = kProjDepth / VEC;  // rows in flight
+// Byte offset of ū[n][k] in one K-major, 128-byte-swizzled operand part [DB/64][BP][128 B].
+__device__ __forceinline__ uint32_t proj_ub_off(int n, int k, int BP) {
+  return static_cast<uint32_t>((k >> 6) * (BP * 128) + n * 128 + ((((k & 63) >> 3) ^ (n & 7)) << 4) + (k & 7) * 2);
+}
+
+// ū rows of the launch's sequences from their slots, VEC columns per thread: kProjDepth / VEC
+// rows in flight; `prep` runs once the first rows are requested, `flush(seq, acc)` receives each
+// sequence's finished sum.
+template <int VEC, typename Prep, typename Flush>
+__device__ __forceinline__ void proj_sum_rows(const float* ubase, size_t ustride, int nrows, const int* rseq,
+                                              const float* wts, int tid, Prep prep, Flush flush) {
+  constexpr int D = kProjDepth / VEC;
   typedef typename std::conditional<VEC == 4, float4, typename std::conditional<VEC == 2, float2, float>::type>::type
       VT;
+  const VT* src = reinterpret_cast<const VT*>(ubase) + tid;
+  const size_t vstride = ustride / VEC;
   float acc[VEC];
 #pragma unroll
   for (int k = 0; k < VEC; ++k) acc[k] = 0.f;
-  int bl = 0;
-  const VT* src = reinterpret_cast<const VT*>(ubase) + tid;
-  const size_t vstride = ustride / VEC;
+  int cur = -1;
+  if (nrows == 0) prep();
+#pragma unroll 1
   for (int c0 = 0; c0 < nrows; c0 += D) {
     VT v[D];
 #pragma unroll
@@ -565,13 +583,12 @@ __device__ __forceinline__ void proj_merge_rows(const float* ubase, size_t ustri
     for (int u = 0; u < D; ++u) {
       const int c = c0 + u;
       if (c >= nrows) break;
-      while (s_beg + c >= s_off[bl + 1]) {  // the previous sequence is complete
+      const int sq = rseq[c];
+      if (sq != cur) {
+        if (cur >= 0) flush(cur, acc);
+        cur = sq;
 #pragma unroll
-        for (int k = 0; k < VEC; ++k) {
-          ub[bl * ubs + VEC * tid + k] = acc[k];
-          acc[k] = 0.f;
-        }
-        ++bl;
+        for (int k = 0; k < VEC; ++k) acc[k] = 0.f;
       }
       const float w = wts[c];
       const float* x = reinterpret_cast<const float*>(&v[u]);
@@ -579,12 +596,7 @@ __device__ __forceinline__ void proj_merge_rows(const float* ubase, size_t ustri
       for (int k = 0; k < VEC; ++k) acc[k] = fmaf(w, x[k], acc[k]);
     }
   }
-  if (nrows > 0) {
-#pragma unroll
-    for (int k = 0; k < VEC; ++k) ub[bl * ubs + VEC * tid + k] = acc[k];
-  } else {
-    prep();
-  }
+  if (cur >= 0) flush(cur, acc);
 }
 
 template <int DHB, int MT>
@@ -593,28 +605,31 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   extern __shared__ uint8_t psm_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(psm_raw) + 1023) & ~uintptr_t(1023));
   constexpr int DH = 64 * DHB;
-  constexpr int NT = DH / 8;                  // 8-column output tiles of a head
-  constexpr int TPW = MT * NT / kProjWarps;   // output tiles per warp
-  static_assert(TPW >= 1 && TPW * kProjWarps == MT * NT, "tiles must split evenly over the warps");
+  constexpr int BP = 16 * MT;                         // N of the projection MMA
+  constexpr uint32_t kTmemCols = BP <= 32 ? 32 : 64;  // fp32 accumulator columns
   const int h = blockIdx.x, r = blockIdx.y;
   const int DB = p.d / p.ndb, c0 = r * DB;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nb = p.nb, b0 = p.b_begin, WS = p.ws;
   const ProjSmem L = proj_smem_layout(DB, DH, nb, p.ndb, WS, p.max_items);
   uint8_t* wring = sm + L.w;
-  float* ub = reinterpret_cast<float*>(sm + L.ub);
-  float* wts = reinterpret_cast<float*>(sm + L.wts);
-  float* ls = reinterpret_cast<float*>(sm + L.ls);
-  int* s_off = reinterpret_cast<int*>(sm + L.soff);
+  uint8_t* ubhi = sm + L.ub;
+  uint8_t* ublo = ubhi + static_cast<uint32_t>(DB) * BP * 2u;
   float* part = reinterpret_cast<float*>(sm + L.part);
   float* recv = reinterpret_cast<float*>(sm + L.recv);
+  float* wts = reinterpret_cast<float*>(sm + L.wts);
+  float* ls = reinterpret_cast<float*>(sm + L.ls);
+  int* rseq = reinterpret_cast<int*>(sm + L.rseq);
+  int* s_off = reinterpret_cast<int*>(sm + L.soff);
   uint64_t* wfull = reinterpret_cast<uint64_t*>(sm + L.bars);
-  uint64_t* wempty = wfull + WS;  // every warp is done with the stage
-  const int ubs = static_cast<int>(L.ubs), per = static_cast<int>(L.per);
+  uint64_t* wempty = wfull + WS;  // the MMAs of the stage completed
+  uint64_t* accbar = wempty + WS;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L.slot);
+  int* fail = reinterpret_cast<int*>(sm + L.slot + 4);
   const int nws = DB / kProjWRows;  // W_KV stages of this block
   constexpr uint32_t kWStageBytes = kProjWRows * DH * 2u;
 
-  int w_issued = 0;  // thread 0 issues every W_KV copy
+  int w_issued = 0;  // thread 0 issues every W_KV copy and MMA
   auto issue_w = [&](int st) {  // W_KV rows c0 + 64 st .., head-h columns, into ring stage st % WS
     uint8_t* dst = wring + (st % WS) * kWStageBytes;
     uint64_t* bar = &wfull[st % WS];
@@ -627,17 +642,31 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   };
 
   // ---- before the split kernel's results exist
-  if (tid == 0) {
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  } else if (warp == 1 && lane == 0) {
     for (int s = 0; s < WS; ++s) {
       mbar_init(&wfull[s], 1);
-      mbar_init(&wempty[s], kProjWarps);
+      mbar_init(&wempty[s], 1);
     }
+    mbar_init(accbar, 1);
+    *fail = 0;
     fence_barrier_init();
+  }
+  {
+    uint4* z = reinterpret_cast<uint4*>(ubhi);  // operand rows of absent sequences stay zero
+    const int n16 = static_cast<int>(2u * static_cast<uint32_t>(DB) * BP * 2u / 16u);
+    for (int i = tid; i < n16; i += kProjThreads) z[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (tid == 0) {
     tma_prefetch_desc(&wmap);
     for (int st = 0; st < min(WS, nws); ++st) issue_w(st);
   }
-  const int Bp = (nb + 15) & ~15;
-  for (int i = tid; i < Bp * ubs; i += kProjThreads) ub[i] = 0.f;
   if (p.ndb > 1) cluster_arrive_relaxed();
   pdl_wait_primary();
   pdl_launch_dependents();
@@ -650,13 +679,14 @@ __global__ void __launch_bounds__(kProjThreads, 1)
   __syncthreads();
   const int s_beg = s_off[0], nrows = s_off[nb] - s_beg;
 
-  // ---- m and l of every slot (one load each, all in flight together)
+  // ---- m and l of every slot (one load each, all in flight together) and each slot's sequence
   for (int c = tid; c < nrows; c += kProjThreads) {
     wts[c] = __ldcg(p.m + static_cast<size_t>(s_beg + c) * p.H + h);
     ls[c] = __ldcg(p.l + static_cast<size_t>(s_beg + c) * p.H + h);
   }
-  // merge weights 2^(m_c - M) / Σ_c' 2^(m_c' - M) l_c', one warp per sequence, from shared memory;
-  // run by proj_merge_rows once its first rows are in flight
+  for (int bl = warp; bl < nb; bl += kProjWarps)
+    for (int c = s_off[bl] - s_beg + lane; c < s_off[bl + 1] - s_beg; c += 32) rseq[c] = bl;
+  // merge weights, one warp per sequence, from shared memory; run once the first rows are in flight
   auto weights = [&]() {
     __syncthreads();
     for (int bl = warp; bl < nb; bl += kProjWarps) {
@@ -678,106 +708,118 @@ __global__ void __launch_bounds__(kProjThreads, 1)
     __syncthreads();
   };
 
-  // ---- ū[b, block] = Σ_c w_c U_c[block]
+  // ---- ū[b, block] = Σ_c w_c U_c[block]; each finished sequence becomes the bf16 high and low
+  // operand rows
   {
     const float* ubase = p.U + (static_cast<size_t>(s_beg) * p.H + h) * p.d + c0;
     const size_t ustride = static_cast<size_t>(p.H) * p.d;  // floats between slots
-    if (DB == 1024) proj_merge_rows<4>(ubase, ustride, nrows, s_beg, s_off, wts, ub, ubs, tid, weights);
-    else if (DB == 512) proj_merge_rows<2>(ubase, ustride, nrows, s_beg, s_off, wts, ub, ubs, tid, weights);
-    else proj_merge_rows<1>(ubase, ustride, nrows, s_beg, s_off, wts, ub, ubs, tid, weights);
+    auto flush = [&](int seq, const float* acc, int vec) {
+      for (int k = 0; k < vec; ++k) {
+        const int col = vec * tid + k;
+        const __nv_bfloat16 hi = __float2bfloat16_rn(acc[k]);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(acc[k] - __bfloat162float(hi));
+        const uint32_t off = proj_ub_off(seq, col, BP);
+        *reinterpret_cast<__nv_bfloat16*>(ubhi + off) = hi;
+        *reinterpret_cast<__nv_bfloat16*>(ublo + off) = lo;
+      }
+    };
+    if (DB == 1024)
+      proj_sum_rows<4>(ubase, ustride, nrows, rseq, wts, tid, weights,
+                       [&](int sq, const float (&a)[4]) { flush(sq, a, 4); });
+    else if (DB == 512)
+      proj_sum_rows<2>(ubase, ustride, nrows, rseq, wts, tid, weights,
+                       [&](int sq, const float (&a)[2]) { flush(sq, a, 2); });
+    else
+      proj_sum_rows<1>(ubase, ustride, nrows, rseq, wts, tid, weights,
+                       [&](int sq, const float (&a)[1]) { flush(sq, a, 1); });
   }
+  fence_proxy_async_smem();  // the operand is read by the tensor cores (async proxy)
   __syncthreads();
 
-  // ---- o_r = ū[:, block] · W_KV[block, h-cols] on mma.sync, W_KV through the ring
-  float acc[TPW][4];
-#pragma unroll
-  for (int i = 0; i < TPW; ++i)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) acc[i][e] = 0.f;
-  const int g = lane >> 2, tq = lane & 3;
-  bool ok = true;
-  int w_done = 0;  // stages thread 0 has seen released by every warp
-  for (int st = 0; st < nws; ++st) {
-    const bool got = __all_sync(0xffffffffu, mbar_wait(&wfull[st % WS], static_cast<uint32_t>(st / WS) & 1u,
-                                                        p.status));
-    if (!got) {
-      ok = false;
-      break;
-    }
-    {
-      const uint32_t wbase = smem_u32(wring + (st % WS) * kWStageBytes);
-#pragma unroll
-      for (int kk = 0; kk < kProjWRows / 16; ++kk) {
-        const int k0 = st * kProjWRows + kk * 16;  // column of ū
-        const int wrow = kk * 16 + (lane & 15);    // row within the stage
-        int mt_prev = -1;
-        uint32_t ahi[4], alo[4];
-#pragma unroll
-        for (int i = 0; i < TPW; ++i) {
-          const int t = warp + kProjWarps * i;
-          const int mt = t / NT, nt = t - mt * NT;
-          if (mt != mt_prev) {
-            mt_prev = mt;
-            const float* a = ub + (mt * 16 + g) * ubs + k0 + 2 * tq;
-            const float2 xs[4] = {*reinterpret_cast<const float2*>(a), *reinterpret_cast<const float2*>(a + 8 * ubs),
-                                  *reinterpret_cast<const float2*>(a + 8),
-                                  *reinterpret_cast<const float2*>(a + 8 * ubs + 8)};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const __nv_bfloat16 h0 = __float2bfloat16_rn(xs[e].x), h1 = __float2bfloat16_rn(xs[e].y);
-              ahi[e] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
-                       (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
-              alo[e] = pack_bf16x2(xs[e].x - __bfloat162float(h0), xs[e].y - __bfloat162float(h1));
-            }
-          }
-          uint32_t b0f, b1f;
-          ldmatrix_x2_trans(wbase + ((nt >> 3) * kProjWRows + wrow) * 128 + (((nt & 7) ^ (wrow & 7)) << 4), b0f,
-                            b1f);
-          mma_16816_bf16(acc[i], ahi, b0f, b1f);
-          mma_16816_bf16(acc[i], alo, b0f, b1f);
-        }
-      }
-    }
-    // release the stage; thread 0 refills it once every warp has
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&wempty[st % WS]);
-    if (tid == 0 && st + WS < nws) {
-      if (!mbar_wait(&wempty[st % WS], static_cast<uint32_t>(st / WS) & 1u, p.status)) {
+  // ---- o_r = W_KV[block, h-cols]^T · ū^T on tcgen05
+  if (tid == 0) {
+    const uint32_t idesc = idesc_bf16_f32(static_cast<uint32_t>(DH), static_cast<uint32_t>(BP), 1u, 0u);
+    const uint32_t wbase = smem_u32(wring), hib = smem_u32(ubhi), lob = smem_u32(ublo);
+    const int lag = min(3, WS - 1);
+    bool ok = true;
+    int done = 0;  // stages whose copies were waited for
+    for (int st = 0; st < nws; ++st) {
+      if (!mbar_wait(&wfull[st % WS], static_cast<uint32_t>(st / WS) & 1u, p.status)) {
         ok = false;
         break;
       }
-      w_done = st + 1;
-      issue_w(st + WS);
+      done = st + 1;
+      tc_fence_after();
+      const uint32_t ws_ = wbase + (st % WS) * kWStageBytes;
+#pragma unroll
+      for (int kk = 0; kk < kProjWRows / 16; ++kk) {
+        // A: MN-major (d_h contiguous), 64-column blocks 64 rows x 128 B (8 KB) apart, 8-row groups
+        // 1024 B apart, a 16-row step is 2 KB. B: K-major rows of 128 B, 8-row groups 1024 B apart,
+        // a 16-column step is 32 B, a 64-column chunk is BP x 128 B.
+        const uint64_t ad = smem_desc(ws_ + kk * 2048, kProjWRows * 128, 1024, kLayoutSW128);
+        const uint32_t boff = st * (BP * 128) + kk * 32;
+        umma_f16(tmem, ad, smem_desc(hib + boff, 16, 1024, kLayoutSW128), idesc, (st > 0 || kk > 0) ? 1u : 0u);
+        umma_f16(tmem, ad, smem_desc(lob + boff, 16, 1024, kLayoutSW128), idesc, 1u);
+      }
+      umma_commit(&wempty[st % WS]);
+      // refill the stage used `lag` stages ago: its MMAs have completed by now, so the refill does
+      // not wait on the tensor pipe (stage st - lag + WS is needed only lag - WS stages later)
+      const int jw = st - lag;
+      if (jw >= 0 && jw + WS < nws) {
+        if (!mbar_wait(&wempty[jw % WS], static_cast<uint32_t>(jw / WS) & 1u, p.status)) {
+          ok = false;
+          break;
+        }
+        issue_w(jw + WS);
+      }
+    }
+    umma_commit(accbar);  // also after a failure: covers every MMA issued
+    if (!ok) {
+      *fail = 1;
+      // copies still landing in this CTA's shared memory must complete before it exits
+      for (int st = done; st < w_issued; ++st)
+        mbar_wait(&wfull[st % WS], static_cast<uint32_t>(st / WS) & 1u, p.status);
     }
   }
-  ok = __syncthreads_and(ok);
-  if (!ok && tid == 0) {
-    // copies still landing in this CTA's shared memory must complete before it exits
-    for (int st = w_done; st < w_issued; ++st)
-      mbar_wait(&wfull[st % WS], static_cast<uint32_t>(st / WS) & 1u, p.status);
-  }
+  __syncwarp();
+  bool ok = mbar_wait(accbar, 0u, p.status);
+  ok = __syncthreads_and(ok) && *fail == 0;
+  tc_fence_after();
+  // accumulator row n (output column n of the head) holds the BP sequences' values
+  if (warp < 4) {
+    const bool has_row = DH == 128 || lane < 16;  // M = 64: lanes 16..31 of a quarter are unused
+    const int n = DH == 128 ? warp * 32 + lane : warp * 16 + lane;
 #pragma unroll
-  for (int i = 0; i < TPW; ++i) {
-    const int t = warp + kProjWarps * i;
-    const int mt = t / NT, nt = t - mt * NT;
-    const int row = mt * 16 + g, col = nt * 8 + 2 * tq;
-    if (row < nb) *reinterpret_cast<float2*>(part + row * DH + col) = make_float2(acc[i][0], acc[i][1]);
-    if (row + 8 < nb) *reinterpret_cast<float2*>(part + (row + 8) * DH + col) = make_float2(acc[i][2], acc[i][3]);
+    for (int cb = 0; cb < BP; cb += 16) {
+      float v[16];
+      tmem_ld16(tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(cb), v);
+      tmem_wait_ld();
+      if (has_row) {
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          if (cb + e < nb) part[(cb + e) * DH + n] = ok ? v[e] : 0.f;
+      }
+    }
   }
+  tc_fence_before();
   __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
 
   // ---- sum the NDB products: push each element to its owner CTA, then add in a fixed order
   const int n_out = nb * DH;
   if (p.ndb == 1) {
     for (int e = tid; e < n_out; e += kProjThreads)
-      p.out[static_cast<size_t>(b0 + e / DH) * p.d + h * DH + e % DH] = ok ? part[e] : 0.f;
+      p.out[static_cast<size_t>(b0 + e / DH) * p.d + h * DH + e % DH] = part[e];
     return;
   }
   cluster_wait();  // every CTA of the cluster is running
   const uint32_t recv_base = smem_u32(recv);
+  const int per = static_cast<int>(L.per);
   for (int e = tid; e < n_out; e += kProjThreads)
-    st_cluster_f32(mapa_shared(recv_base + 4u * static_cast<uint32_t>(r * per + e / p.ndb), e % p.ndb),
-                   ok ? part[e] : 0.f);
+    st_cluster_f32(mapa_shared(recv_base + 4u * static_cast<uint32_t>(r * per + e / p.ndb), e % p.ndb), part[e]);
   cluster_sync();  // pushes visible; nobody touches a peer's shared memory after this
   for (int s2 = tid; s2 < per; s2 += kProjThreads) {
     const int e = s2 * p.ndb + r;
@@ -869,8 +911,6 @@ struct ProjConfig {
   uint32_t smem;
 };
 
-constexpr int kProjMaxSeqs = 64;  // sequences per launch: MT <= 4 tiles of 16
-
 template <int DHB, int MT>
 int proj_resident_clusters(int ndb, uint32_t smem, int H) {
   cudaLaunchConfig_t cfg = {};
@@ -906,42 +946,48 @@ int proj_resident(int dhb, int mt, int ndb, uint32_t smem, int H) {
   return 0;
 }
 
-// Projection merge for bf16 W_KV and d_h = 64 or 128. NDB (1..8, DB = d/NDB a multiple of 64
-// and at most 1024) is chosen so that the H x NDB CTAs run in one wave with as many CTAs as
-// possible (the fewest blocks on a tie); the U ring holds about 64 KB of rows in flight.
+// Projection merge for bf16 W_KV and d_h = 64 or 128. Up to 64 sequences per launch (fewer when
+// the operand does not fit); NDB (1..8, DB = d/NDB of 256, 512 or 1024 columns) is chosen so that
+// the H x NDB CTAs run in one wave with as many CTAs as possible (the fewest blocks on a tie); the
+// W_KV ring gets as many stages as fit (the whole block when it does), at least two.
 bool pick_proj_uncached(int B, int d, int H, int max_items, ProjConfig* c) {
   const int d_h = d / H;
   if (d_h != 64 && d_h != 128) return false;
-  c->nb_max = kProjMaxSeqs;
-  const int nb = std::min(B, kProjMaxSeqs);
-  const int mt = (nb + 15) / 16;
   const uint32_t optin = static_cast<uint32_t>(max_smem_optin());
-  int best = 0, best_ctas = -1, best_ws = 0;
-  uint32_t best_smem = 0;
-  for (int ndb = 1; ndb <= 8; ++ndb) {
-    if (d % ndb) continue;
-    const int DB = d / ndb;
-    if (DB != 256 && DB != 512 && DB != 1024) continue;
-    // as many W_KV stages as fit (the whole block when it does), at least two
-    int ws = std::min(kProjMaxWStages, DB / kProjWRows);
-    uint32_t sm = proj_smem_layout(DB, d_h, nb, ndb, ws, max_items).total;
-    while (sm > optin && ws > 2) sm = proj_smem_layout(DB, d_h, nb, ndb, --ws, max_items).total;
-    if (sm > optin) continue;
-    const int fit = proj_resident(d_h / 64, mt, ndb, sm, H);  // clusters resident at once
-    if (fit <= 0) continue;
-    const int score = H <= fit ? H * ndb : 0;  // CTAs, when all of them run in one wave
-    if (score > best_ctas) {
-      best = ndb;
-      best_ctas = score;
-      best_ws = ws;
-      best_smem = sm;
+  for (int nb_max : {64, 32, 16}) {
+    const int nb = std::min(B, nb_max);
+    const int mt = (nb + 15) / 16;
+    int best = 0, best_ctas = -1, best_ws = 0;
+    uint32_t best_smem = 0;
+    for (int ndb = 1; ndb <= 8; ++ndb) {
+      if (d % ndb) continue;
+      const int DB = d / ndb;
+      if (DB != 256 && DB != 512 && DB != 1024) continue;
+      int ws = std::min(kProjMaxWStages, DB / kProjWRows);
+      uint32_t sm = proj_smem_layout(DB, d_h, nb, ndb, ws, max_items).total;
+      while (sm > optin && ws > 2) sm = proj_smem_layout(DB, d_h, nb, ndb, --ws, max_items).total;
+      if (sm > optin) continue;
+      const int fit = proj_resident(d_h / 64, mt, ndb, sm, H);  // clusters resident at once
+      if (fit <= 0) continue;
+      const int score = H <= fit ? H * ndb : 0;  // CTAs, when all of them run in one wave
+      if (score > best_ctas) {
+        best = ndb;
+        best_ctas = score;
+        best_ws = ws;
+        best_smem = sm;
+      }
     }
+    if (best == 0) {
+      if (nb < nb_max) return false;  // a smaller launch would not help
+      continue;
+    }
+    c->ndb = best;
+    c->ws = best_ws;
+    c->nb_max = nb_max;
+    c->smem = best_smem;
+    return true;
   }
-  if (best == 0) return false;
-  c->ndb = best;
-  c->ws = best_ws;
-  c->smem = best_smem;
-  return true;
+  return false;
 }
 
 // pick_proj_uncached memoised per (device, shape): it queries the occupancy API.
