@@ -947,9 +947,10 @@ int proj_resident(int dhb, int mt, int ndb, uint32_t smem, int H) {
 }
 
 // Projection merge for bf16 W_KV and d_h = 64 or 128. Up to 64 sequences per launch (fewer when
-// the operand does not fit); NDB (1..8, DB = d/NDB of 256, 512 or 1024 columns) is chosen so that
-// the H x NDB CTAs run in one wave with as many CTAs as possible (the fewest blocks on a tie); the
-// W_KV ring gets as many stages as fit (the whole block when it does), at least two.
+// the operand does not fit). NDB (1..8, DB = d/NDB of 256, 512 or 1024 columns) and the W_KV ring
+// depth are chosen so that the H x NDB CTAs run in one wave with as many CTAs as possible (a
+// shallower ring that lets two CTAs share an SM counts), then the deepest ring, then the fewest
+// blocks.
 bool pick_proj_uncached(int B, int d, int H, int max_items, ProjConfig* c) {
   const int d_h = d / H;
   if (d_h != 64 && d_h != 128) return false;
@@ -963,18 +964,20 @@ bool pick_proj_uncached(int B, int d, int H, int max_items, ProjConfig* c) {
       if (d % ndb) continue;
       const int DB = d / ndb;
       if (DB != 256 && DB != 512 && DB != 1024) continue;
-      int ws = std::min(kProjMaxWStages, DB / kProjWRows);
-      uint32_t sm = proj_smem_layout(DB, d_h, nb, ndb, ws, max_items).total;
-      while (sm > optin && ws > 2) sm = proj_smem_layout(DB, d_h, nb, ndb, --ws, max_items).total;
-      if (sm > optin) continue;
-      const int fit = proj_resident(d_h / 64, mt, ndb, sm, H);  // clusters resident at once
-      if (fit <= 0) continue;
-      const int score = H <= fit ? H * ndb : 0;  // CTAs, when all of them run in one wave
-      if (score > best_ctas) {
-        best = ndb;
-        best_ctas = score;
-        best_ws = ws;
-        best_smem = sm;
+      int last_fit = -1;
+      for (int ws = std::min(kProjMaxWStages, DB / kProjWRows); ws >= 2; --ws) {
+        const uint32_t sm = proj_smem_layout(DB, d_h, nb, ndb, ws, max_items).total;
+        if (sm > optin) continue;
+        const int fit = proj_resident(d_h / 64, mt, ndb, sm, H);  // clusters resident at once
+        if (fit <= 0 || fit == last_fit) continue;  // a shallower ring only helps if more CTAs fit
+        last_fit = fit;
+        const int score = H <= fit ? H * ndb : 0;  // CTAs, when all of them run in one wave
+        if (score > best_ctas) {
+          best = ndb;
+          best_ctas = score;
+          best_ws = ws;
+          best_smem = sm;
+        }
       }
     }
     if (best == 0) {
