@@ -10,13 +10,24 @@
 //     o_i = softmax(q_i · K_{<=p_i}^T / sqrt(d_h)) · V_{<=p_i}
 // per head, p_i the position of query i (its own key included).
 //
-// This kernel is the attention part, flash-attention style on warp-level
-// tensor-core MMAs (mma.sync m16n8k16, bf16 in, fp32 accumulation): a CTA owns
-// 64 queries of one head of one sequence (16 per warp), streams 64-row tiles
-// of K and V (TMA, 128-byte swizzle, 3-stage ring, bounded waits), computes
-// S = Q·K^T, keeps a running max and sum per query row in registers, and adds
-// P·V into register accumulators; the score accumulators are reused as the A
-// operand of P·V without leaving registers.
+// This kernel is the attention part, flash-attention style on tcgen05 tensor cores: a CTA owns
+// 128 queries of one head of one sequence and walks the 64-key tiles up to its last query's
+// position.
+//   warp 0     TMA producer: the Q tile once, then K and V tiles (64 rows x d_h, 128-byte swizzle,
+//              K and V on separate barriers) through a ring of 5 (d_h = 128) or 8 stages
+//   warp 1     tcgen05.mma issuer: S = Q·K^T (M = 128 queries, N = 64 keys, K = d_h) into one of
+//              two 64-column TMEM buffers, so that the next tile's scores are computed while this
+//              tile's softmax runs; O += P·V (M = 128, N = d_h, K = 64 keys) into a third TMEM
+//              region, P read from one of two shared-memory buffers (K-major; the softmax of the
+//              next tile writes the other while this P·V runs) and V in place as the MN-major
+//              operand
+//   warps 4-7  softmax, one query row per thread (TMEM lane = row): the tile's scores, the causal
+//              mask, a running max kept lazily (O is rescaled in TMEM only when a row's max grows by
+//              more than 2^8, so P <= 2^8 stays exact enough in bf16), P in bf16 to shared memory,
+//              the row sums in fp32 registers; at the end o = O / l to global memory.
+// Key rows at or past a sequence's length are scratch in the V buffer: their rows of the last
+// tile are zeroed in shared memory before the P·V MMA (a masked score's p = 0 never meets a
+// non-finite value).
 #include <cuda_bf16.h>
 
 #include "ptx.cuh"
@@ -25,10 +36,10 @@ namespace slim {
 
 namespace {
 
-constexpr int kPQ = 64;       // queries per CTA
-constexpr int kPK = 64;       // keys per tile
-constexpr int kPStages = 3;
-constexpr int kPThreads = 128;
+constexpr int kPQ = 128;  // queries per CTA (the MMA's M)
+constexpr int kPK = 64;   // keys per tile
+constexpr int kPThreads = 256;
+constexpr float kPLazyLog2 = 8.f;
 
 struct PrefillAttnParams {
   float* out;           // [B][n][d]
@@ -39,40 +50,38 @@ struct PrefillAttnParams {
   float scale_log2;
 };
 
-__host__ __device__ inline uint32_t pa_tile_bytes(int dhb) { return kPK * 128u * dhb; }
+__host__ __device__ inline int pa_stages(int dhb) { return dhb == 2 ? 4 : 8; }
+__host__ __device__ inline uint32_t pa_q_bytes(int dhb) { return 128u * 128u * dhb; }  // 128 queries x d_h bf16
+__host__ __device__ inline uint32_t pa_kv_bytes(int dhb) { return 64u * 128u * dhb; }  // 64 keys x d_h bf16
 __host__ __device__ inline uint32_t pa_smem_bytes(int dhb) {
-  return pa_tile_bytes(dhb) /*Q*/ + kPStages * 2u * pa_tile_bytes(dhb) /*K, V*/ + (1u + kPStages) * 8u + 1024u;
-}
-
-// byte offset of (row r, column c) in a tile of 64 rows x 64·DHB columns: [c / 64 boxes][64 rows][128 B], swizzled
-__device__ __forceinline__ uint32_t pa_off(int r, int c) {
-  return static_cast<uint32_t>((c >> 6) * (kPK * 128) + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4));
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
+  // Q, the K/V ring, two P buffers (128 x 64 bf16), barriers, TMEM slot; slack for 1024-byte alignment
+  return pa_q_bytes(dhb) + pa_stages(dhb) * 2u * pa_kv_bytes(dhb) + 2u * 16384u + 512u + 1024u;
 }
 
 template <int DHB>
-__global__ void __launch_bounds__(kPThreads)
+__global__ void __launch_bounds__(kPThreads, 1)
     prefill_attn_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                         const __grid_constant__ CUtensorMap vmap, const PrefillAttnParams p) {
   extern __shared__ uint8_t pa_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pa_raw) + 1023) & ~uintptr_t(1023));
   constexpr int DH = 64 * DHB;
-  constexpr int NTO = DH / 8;  // 8-column tiles of the output
-  const uint32_t TB = pa_tile_bytes(DHB);
-  uint8_t* qs = sm;
-  uint8_t* kvs = sm + TB;  // [stage][K tile, V tile]
-  uint64_t* qbar = reinterpret_cast<uint64_t*>(sm + TB + kPStages * 2u * TB);
-  uint64_t* full = qbar + 1;
+  constexpr int NS = DHB == 2 ? 4 : 8;
+  const uint32_t TQ = pa_q_bytes(DHB), T = pa_kv_bytes(DHB);
+  uint8_t* qs = sm;  // [DHB boxes][128 rows][128 B]
+  uint8_t* kvs = sm + TQ;  // [stage][K tile, V tile], each [DHB boxes][64 rows][128 B]
+  uint8_t* ps = sm + TQ + NS * 2u * T;  // P: [2 buffers][128 rows][128 B] (64 keys)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ps + 2u * 16384u);
+  uint64_t* qbar = bars;                // Q landed
+  uint64_t* kfull = bars + 1;           // [NS] K of a tile landed
+  uint64_t* vfull = kfull + NS;         // [NS] V of a tile landed
+  uint64_t* kvempty = vfull + NS;       // [NS] the tile's MMAs are done with the stage
+  uint64_t* sfull = kvempty + NS;       // [2] S buffer written
+  uint64_t* sfree = sfull + 2;          // [2] S buffer read by the four softmax warps
+  uint64_t* pready = sfree + 2;         // [2] P buffer written (and O rescaled) by the four softmax warps
+  uint64_t* pfree = pready + 2;         // [2] the P·V MMA that read the buffer completed
+  uint64_t* ofull = pfree + 2;          // the last P·V MMA completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ofull + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, tq = lane & 3;
 
   // heaviest query tiles (the last ones) first
   const int nqt = (p.n + kPQ - 1) / kPQ;
@@ -89,166 +98,234 @@ __global__ void __launch_bounds__(kPThreads)
   const int last_key = pos0 + min(q0 + kPQ, p.n) - 1;  // largest position any query here attends
   const int nkt = last_key / kPK + 1;
 
-  int issued = 0;
-  auto issue = [&](int j) {  // K and V rows 64 j .. of this head into stage j % kPStages
-    uint8_t* dst = kvs + (j % kPStages) * 2u * TB;
-    uint64_t* bar = &full[j % kPStages];
-    mbar_arrive_expect_tx(bar, 2u * TB);
-    const int y = static_cast<int>(static_cast<int64_t>(b) * p.cap + j * kPK);
-#pragma unroll
-    for (int i = 0; i < DHB; ++i) {
-      tma_load_2d(dst + i * (kPK * 128), &kmap, h * DH + 64 * i, y, bar, l2_policy_evict_last());
-      tma_load_2d(dst + TB + i * (kPK * 128), &vmap, h * DH + 64 * i, y, bar, l2_policy_evict_last());
-    }
-    ++issued;
-  };
-  if (threadIdx.x == 0) {
+  if (warp == 0 && lane == 0) {
     mbar_init(qbar, 1);
-    for (int s = 0; s < kPStages; ++s) mbar_init(&full[s], 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&kfull[s], 1);
+      mbar_init(&vfull[s], 1);
+      mbar_init(&kvempty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sfull[i], 1);
+      mbar_init(&sfree[i], 4);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&pready[i], 4);
+      mbar_init(&pfree[i], 1);
+    }
+    mbar_init(ofull, 1);
     fence_barrier_init();
-    tma_prefetch_desc(&qmap);
-    tma_prefetch_desc(&kmap);
-    tma_prefetch_desc(&vmap);
-    mbar_arrive_expect_tx(qbar, TB);
-#pragma unroll
-    for (int i = 0; i < DHB; ++i)
-      tma_load_2d(qs + i * (kPK * 128), &qmap, h * DH + 64 * i, b * p.n + q0, qbar, l2_policy_evict_first());
-    for (int j = 0; j < min(kPStages, nkt); ++j) issue(j);
+  } else if (warp == 1) {
+    tmem_alloc(tmem_slot, 256);
+    tmem_relinquish();
   }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem_o = tmem + 128u;  // S buffers at columns 0 and 64
 
-  float o[NTO][4];
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&qmap);
+      tma_prefetch_desc(&kmap);
+      tma_prefetch_desc(&vmap);
+      mbar_arrive_expect_tx(qbar, TQ);
 #pragma unroll
-  for (int i = 0; i < NTO; ++i)
+      for (int i = 0; i < DHB; ++i)
+        tma_load_2d(qs + i * 16384, &qmap, h * DH + 64 * i, b * p.n + q0, qbar, l2_policy_evict_first());
+      int j = 0;
+      for (; j < nkt; ++j) {
+        const int s = j % NS;
+        if (j >= NS && !mbar_wait(&kvempty[s], static_cast<uint32_t>((j / NS) & 1) ^ 1u, p.status)) break;
+        uint8_t* dst = kvs + s * 2u * T;
+        const int y = static_cast<int>(static_cast<int64_t>(b) * p.cap + j * kPK);
+        mbar_arrive_expect_tx(&kfull[s], T);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) o[i][e] = 0.f;
-  float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};  // rows g and g + 8 of the warp
-  const int qr0 = q0 + warp * 16 + g;                           // query index of row g
-  const int pr[2] = {pos0 + qr0, pos0 + qr0 + 8};              // their positions
-  const uint32_t qbase = smem_u32(qs);
-  bool ok = mbar_wait(qbar, 0u, p.status);
-  int done = 0;
-  for (int j = 0; j < nkt; ++j) {
-    const int s = j % kPStages;
-    const bool got = ok && mbar_wait(&full[s], static_cast<uint32_t>(j / kPStages) & 1u, p.status);
-    ok = __syncthreads_and(got);
-    if (!ok) break;
-    const uint32_t kb = smem_u32(kvs + s * 2u * TB), vb = kb + TB;
-    if ((j + 1) * kPK > L) {
-      // rows at or past the sequence's length hold no key or value (the V buffer is scratch there):
-      // zero them so that a masked score's p = 0 never meets a non-finite value
-      uint8_t* kt = kvs + s * 2u * TB;
-      const int r0 = L - j * kPK;
-      for (int i = threadIdx.x; i < (kPK - r0) * 8 * DHB; i += kPThreads) {
-        const int r = r0 + i / (8 * DHB), ch = i % (8 * DHB);
-        const uint32_t off = pa_off(r, ch * 8);
-        *reinterpret_cast<uint4*>(kt + off) = make_uint4(0u, 0u, 0u, 0u);
-        *reinterpret_cast<uint4*>(kt + TB + off) = make_uint4(0u, 0u, 0u, 0u);
+        for (int i = 0; i < DHB; ++i)
+          tma_load_2d(dst + i * 8192, &kmap, h * DH + 64 * i, y, &kfull[s], l2_policy_evict_last());
+        mbar_arrive_expect_tx(&vfull[s], T);
+#pragma unroll
+        for (int i = 0; i < DHB; ++i)
+          tma_load_2d(dst + T + i * 8192, &vmap, h * DH + 64 * i, y, &vfull[s], l2_policy_evict_last());
       }
-      fence_proxy_async_smem();  // these writes come before the stage's next TMA fill
-      __syncthreads();
-    }
-    // S = Q·K^T for the warp's 16 queries x 64 keys
-    float sc[8][4];
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) sc[nt][e] = 0.f;
-#pragma unroll
-    for (int ks = 0; ks < DH / 16; ++ks) {
-      uint32_t a[4];
-      {
-        const int r = warp * 16 + (lane & 15), c = ks * 16 + (lane >> 4) * 8;
-        ldsm_x4(qbase + pa_off(r, c), a[0], a[1], a[2], a[3]);
-      }
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-        uint32_t b0, b1;
-        const int r = nt * 8 + (lane & 7), c = ks * 16 + ((lane >> 3) & 1) * 8;
-        ldsm_x2(kb + pa_off(r, c), b0, b1);
-        mma_16816_bf16(sc[nt], a, b0, b1);
+      // every issued copy lands before the CTA exits
+      mbar_wait(qbar, 0u, p.status);
+      for (int t = max(0, j - NS); t < j; ++t) {
+        mbar_wait(&kfull[t % NS], static_cast<uint32_t>(t / NS) & 1u, p.status);
+        mbar_wait(&vfull[t % NS], static_cast<uint32_t>(t / NS) & 1u, p.status);
       }
     }
-    // causal mask, running max and sum (log2 domain), P in place
-    const int k0 = j * kPK;
-    float mx[2] = {-INFINITY, -INFINITY};
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16_f32(kPQ, kPK, 0u, 0u);
+      const uint32_t idesc_o = idesc_bf16_f32(kPQ, DH, 0u, 1u);
+      const uint32_t qb = smem_u32(qs), kvb = smem_u32(kvs), pb = smem_u32(ps);
+      bool ok = mbar_wait(qbar, 0u, p.status);
+      auto issue_s = [&](int j) {
+        const int s = j % NS, sb = j & 1;
+        if (!mbar_wait(&kfull[s], static_cast<uint32_t>(j / NS) & 1u, p.status)) return false;
+        if (j >= 2 && !mbar_wait(&sfree[sb], static_cast<uint32_t>((j - 2) / 2) & 1u, p.status)) return false;
+        tc_fence_after();
+        const uint32_t kb = kvb + s * 2u * T;
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
+        for (int kk = 0; kk < DH / 16; ++kk) {
+          // Q and K both K-major (d_h contiguous): 64-column boxes 16 KB (Q) or 8 KB (K) apart, 8-row
+          // groups 1024 B apart, a 16-column step is 32 B into the swizzled row
+          const uint32_t cin = (kk & 3) * 32u;
+          umma_f16(tmem + static_cast<uint32_t>(sb * kPK),
+                   smem_desc(qb + (kk >> 2) * 16384u + cin, 16, 1024, kLayoutSW128),
+                   smem_desc(kb + (kk >> 2) * 8192u + cin, 16, 1024, kLayoutSW128), idesc_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&sfull[sb]);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int j = 0; ok && j < nkt; ++j) {
+        if (j + 1 < nkt && !issue_s(j + 1)) {
+          ok = false;
+          break;
+        }
+        if (!mbar_wait(&pready[j & 1], static_cast<uint32_t>(j / 2) & 1u, p.status) ||
+            !mbar_wait(&vfull[j % NS], static_cast<uint32_t>(j / NS) & 1u, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t vb = kvb + (j % NS) * 2u * T + T;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int key = k0 + nt * 8 + 2 * tq + (e & 1);
-        const int rr = e >> 1;
-        const float v = key <= pr[rr] ? sc[nt][e] * p.scale_log2 : -INFINITY;
-        sc[nt][e] = v;
-        mx[rr] = fmaxf(mx[rr], v);
+        for (int kk = 0; kk < kPK / 16; ++kk) {
+          // P K-major (keys contiguous, one 64-key box); V MN-major (d_h contiguous): 64-column
+          // blocks 8 KB apart, 8-key groups 1024 B apart, 16 keys per step
+          umma_f16(tmem_o, smem_desc(pb + (j & 1) * 16384u + kk * 32u, 16, 1024, kLayoutSW128),
+                   smem_desc(vb + kk * 2048u, 8192, 1024, kLayoutSW128), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&kvempty[j % NS]);
+        umma_commit(&pfree[j & 1]);
       }
-    float alpha[2];
-#pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
-      mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 1));
-      mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 2));
-      const float mn = fmaxf(mrow[rr], mx[rr]);
-      alpha[rr] = mn == -INFINITY ? 1.f : exp2f(mrow[rr] - mn);
-      mrow[rr] = mn;
-      lrow[rr] *= alpha[rr];
+      umma_commit(ofull);  // also after a failure: covers every MMA issued
+      mbar_wait(ofull, 0u, p.status);
     }
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int rr = e >> 1;
-        const float pv = mrow[rr] == -INFINITY ? 0.f : exp2f(sc[nt][e] - mrow[rr]);
-        sc[nt][e] = pv;
-        lrow[rr] += pv;
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax warps
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // query row of the tile = TMEM lane
+    const uint32_t lrow = static_cast<uint32_t>(quarter * 32) << 16;
+    const int pos = pos0 + q0 + r;     // position of this row's query
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nkt; ++j) {
+      const int sb = j & 1, s = j % NS;
+      if (!__all_sync(0xffffffffu, mbar_wait(&sfull[sb], static_cast<uint32_t>(j / 2) & 1u, p.status))) {
+        ok = false;
+        break;
       }
+      tc_fence_after();
+      float sc[kPK];
 #pragma unroll
-    for (int i = 0; i < NTO; ++i) {
-      o[i][0] *= alpha[0];
-      o[i][1] *= alpha[0];
-      o[i][2] *= alpha[1];
-      o[i][3] *= alpha[1];
-    }
-    // O += P·V: P (16 x 64) from the score accumulators, V (64 keys x d_h) by transposed loads
+      for (int c = 0; c < kPK / 16; ++c)
+        tmem_ld16(tmem + lrow + static_cast<uint32_t>(sb * kPK + 16 * c), *reinterpret_cast<float(*)[16]>(sc + 16 * c));
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sfree[sb]);
+      // scores in the log2 domain, keys past this query masked
+      const int k0 = j * kPK;
+      float mt = -INFINITY;
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {  // 16 keys at a time
-      uint32_t a[4];
-      a[0] = pack_bf16x2(sc[2 * kk][0], sc[2 * kk][1]);
-      a[1] = pack_bf16x2(sc[2 * kk][2], sc[2 * kk][3]);
-      a[2] = pack_bf16x2(sc[2 * kk + 1][0], sc[2 * kk + 1][1]);
-      a[3] = pack_bf16x2(sc[2 * kk + 1][2], sc[2 * kk + 1][3]);
-#pragma unroll
-      for (int nt = 0; nt < NTO; ++nt) {
-        uint32_t b0, b1;
-        const int r = kk * 16 + (lane & 15), c = nt * 8;
-        ldmatrix_x2_trans(vb + pa_off(r, c), b0, b1);
-        mma_16816_bf16(o[nt], a, b0, b1);
+      for (int c = 0; c < kPK; ++c) {
+        const float v = (k0 + c <= pos) ? sc[c] * p.scale_log2 : -INFINITY;
+        sc[c] = v;
+        mt = fmaxf(mt, v);
       }
+      float alpha = 1.f;
+      if (j == 0 || m == -INFINITY) {
+        m = mt;
+      } else if (mt > m + kPLazyLog2) {
+        alpha = exp2f(m - mt);
+        m = mt;
+        l *= alpha;
+      }
+      // P = 2^(s - m) in bf16 (the row sum adds the rounded values the MMA sees)
+      uint32_t pk[kPK / 2];
+#pragma unroll
+      for (int c = 0; c < kPK / 2; ++c) {
+        const float a = m == -INFINITY ? 0.f : exp2f(sc[2 * c] - m);
+        const float bb = m == -INFINITY ? 0.f : exp2f(sc[2 * c + 1] - m);
+        const __nv_bfloat16 ha = __float2bfloat16_rn(a), hb = __float2bfloat16_rn(bb);
+        l += __bfloat162float(ha) + __bfloat162float(hb);
+        pk[c] = static_cast<uint32_t>(__bfloat16_as_ushort(ha)) | (static_cast<uint32_t>(__bfloat16_as_ushort(hb)) << 16);
+      }
+      // this P buffer was last read by the P·V of tile j - 2
+      const int pbuf = j & 1;
+      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&pfree[pbuf], static_cast<uint32_t>((j - 2) / 2) & 1u, p.status))) {
+        ok = false;
+        break;
+      }
+      if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        // O is rescaled once the previous tile's P·V has completed
+        if (!__all_sync(0xffffffffu, mbar_wait(&pfree[pbuf ^ 1], static_cast<uint32_t>((j - 1) / 2) & 1u, p.status))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int c = 0; c < DH; c += 16) {
+          float v[16];
+          tmem_ld16(tmem_o + lrow + static_cast<uint32_t>(c), v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] *= alpha;
+          tmem_st16(tmem_o + lrow + static_cast<uint32_t>(c), v);
+        }
+        tmem_wait_st();
+      }
+      // P row r: [row][16-byte chunk ^ (row & 7)]
+#pragma unroll
+      for (int c = 0; c < kPK / 8; ++c) {
+        const uint32_t off = static_cast<uint32_t>(pbuf * 16384 + r * 128 + ((c ^ (r & 7)) << 4));
+        *reinterpret_cast<uint4*>(ps + off) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      }
+      // key rows at or past the length in this tile hold no value: zero them in V (thread r < 64
+      // takes key row r, once the tile's V has landed)
+      if (k0 + kPK > L && r < kPK && k0 + r >= L) {
+        if (mbar_wait(&vfull[s], static_cast<uint32_t>(j / NS) & 1u, p.status)) {
+          uint8_t* vrow = kvs + s * 2u * T + T + r * 128;
+#pragma unroll
+          for (int i = 0; i < DHB; ++i)
+#pragma unroll
+            for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(vrow + i * 8192 + c * 16) = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      fence_proxy_async_smem();  // P (and zeroed V rows) are read by the tensor cores
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&pready[pbuf]);
     }
-    done = j + 1;
-    __syncthreads();  // every warp is done with the stage
-    if (threadIdx.x == 0 && j + kPStages < nkt) issue(j + kPStages);
-  }
-  if (!ok && threadIdx.x == 0) {
-    // copies still landing in this CTA's shared memory must complete before it exits
-    mbar_wait(qbar, 0u, p.status);
-    for (int j = done; j < issued; ++j)
-      mbar_wait(&full[j % kPStages], static_cast<uint32_t>(j / kPStages) & 1u, p.status);
-  }
-  // o / l, rows of the warp's queries that exist
-#pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
-    lrow[rr] += __shfl_xor_sync(0xffffffffu, lrow[rr], 1);
-    lrow[rr] += __shfl_xor_sync(0xffffffffu, lrow[rr], 2);
-  }
-#pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
-    const int qi = qr0 + 8 * rr;
-    if (qi >= p.n) continue;
-    const float inv = (ok && lrow[rr] > 0.f) ? 1.f / lrow[rr] : 0.f;
+    // o = O / l
+    const bool got = ok && __all_sync(0xffffffffu, mbar_wait(ofull, 0u, p.status));
+    tc_fence_after();
+    const int qi = q0 + r;
+    const float inv = (got && l > 0.f) ? 1.f / l : 0.f;
     float* dst = p.out + (static_cast<size_t>(b) * p.n + qi) * p.d + h * DH;
+    for (int c = 0; c < DH; c += 16) {
+      float v[16];
+      tmem_ld16(tmem_o + lrow + static_cast<uint32_t>(c), v);
+      tmem_wait_ld();
+      if (qi < p.n) {
 #pragma unroll
-    for (int nt = 0; nt < NTO; ++nt)
-      *reinterpret_cast<float2*>(dst + nt * 8 + 2 * tq) = make_float2(o[nt][2 * rr] * inv, o[nt][2 * rr + 1] * inv);
+        for (int i = 0; i < 16; i += 4)
+          *reinterpret_cast<float4*>(dst + c + i) = make_float4(v[i] * inv, v[i + 1] * inv, v[i + 2] * inv, v[i + 3] * inv);
+      }
+    }
+  }
+  __syncwarp();  // lanes 1..31 of warps 0 and 1 skipped the lane-0 loops
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
   }
 }
 

@@ -78,3 +78,9 @@ def test_prompt_attention_d1024(S):
 def test_prompt_attention_d4096(S):
     """d_h = 128, one sequence of 150 prompt rows."""
     _run(S, 4096, 32, [0], 150, seed=52)
+
+
+def test_prompt_attention_many_key_tiles(S):
+    """d_h = 64, 700 prompt rows after 200 cached ones: up to 8 key tiles of 128 per query tile,
+    both S buffers and the K/V ring reused several times, a ragged last key tile."""
+    _run(S, 1024, 16, [200], 700, seed=53)
