@@ -51,6 +51,14 @@ struct PrefillAttnParams {
 };
 
 __host__ __device__ inline int pa_stages(int dhb) { return dhb == 2 ? 4 : 8; }
+
+// 2^x on the special-function unit (the PTX approximate base-2 exponential; subnormal results flush
+// to zero, which for a softmax weight below 2^-126 is a zero weight).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 __host__ __device__ inline uint32_t pa_q_bytes(int dhb) { return 128u * 128u * dhb; }  // 128 queries x d_h bf16
 __host__ __device__ inline uint32_t pa_kv_bytes(int dhb) { return 64u * 128u * dhb; }  // 64 keys x d_h bf16
 __host__ __device__ inline uint32_t pa_smem_bytes(int dhb) {
@@ -231,33 +239,39 @@ __global__ void __launch_bounds__(kPThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sfree[sb]);
-      // scores in the log2 domain, keys past this query masked
+      // keys past this query masked (only a tile that reaches past the query has any); the scale
+      // is applied with the exponent below (max(s)·scale = max(s·scale) for scale > 0)
       const int k0 = j * kPK;
-      float mt = -INFINITY;
+      if (k0 + kPK - 1 > pos) {
 #pragma unroll
-      for (int c = 0; c < kPK; ++c) {
-        const float v = (k0 + c <= pos) ? sc[c] * p.scale_log2 : -INFINITY;
-        sc[c] = v;
-        mt = fmaxf(mt, v);
+        for (int c = 0; c < kPK; ++c) sc[c] = (k0 + c <= pos) ? sc[c] : -INFINITY;
       }
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int c = 0; c < kPK; ++c) mx[c & 3] = fmaxf(mx[c & 3], sc[c]);
+      const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.scale_log2;
       float alpha = 1.f;
       if (j == 0 || m == -INFINITY) {
         m = mt;
       } else if (mt > m + kPLazyLog2) {
-        alpha = exp2f(m - mt);
+        alpha = ex2_approx(m - mt);
         m = mt;
         l *= alpha;
       }
-      // P = 2^(s - m) in bf16 (the row sum adds the rounded values the MMA sees)
+      // P = 2^(s·scale - m) in bf16; the row sum adds the rounded values the MMA sees
       uint32_t pk[kPK / 2];
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      const float nm = m == -INFINITY ? 0.f : -m;
 #pragma unroll
       for (int c = 0; c < kPK / 2; ++c) {
-        const float a = m == -INFINITY ? 0.f : exp2f(sc[2 * c] - m);
-        const float bb = m == -INFINITY ? 0.f : exp2f(sc[2 * c + 1] - m);
-        const __nv_bfloat16 ha = __float2bfloat16_rn(a), hb = __float2bfloat16_rn(bb);
-        l += __bfloat162float(ha) + __bfloat162float(hb);
-        pk[c] = static_cast<uint32_t>(__bfloat16_as_ushort(ha)) | (static_cast<uint32_t>(__bfloat16_as_ushort(hb)) << 16);
+        const float a = ex2_approx(fmaf(sc[2 * c], p.scale_log2, nm));
+        const float bb = ex2_approx(fmaf(sc[2 * c + 1], p.scale_log2, nm));
+        const __nv_bfloat162 hv = __floats2bfloat162_rn(a, bb);
+        const float2 f = __bfloat1622float2(hv);
+        ls[c & 3] += f.x + f.y;
+        pk[c] = *reinterpret_cast<const uint32_t*>(&hv);
       }
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       // this P buffer was last read by the P·V of tile j - 2
       const int pbuf = j & 1;
       if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&pfree[pbuf], static_cast<uint32_t>((j - 2) / 2) & 1u, p.status))) {
