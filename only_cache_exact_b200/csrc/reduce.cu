@@ -12,9 +12,11 @@
 //     B·H CTAs in one wave; the head slice of W_KV is held whole in shared memory.
 //   * merge_proj_kernel  bf16 W_KV with d_h = 64 or 128, any batch: one CTA per
 //     (head, block of d rows), all CTAs in one wave, clusters along the blocks.
-//     The partial rows are read with many loads in flight per thread, W_KV
-//     through a ring of TMA tiles; the projection runs on mma.sync; the blocks'
-//     products are summed in a fixed order through distributed shared memory.
+//     The partial rows are read with many loads in flight per thread and summed
+//     into a bf16 high/low tcgen05 operand; W_KV streams through a ring of TMA
+//     tiles and the projection runs on tcgen05 with a TMEM accumulator; the
+//     blocks' products are summed in a fixed order through distributed shared
+//     memory.
 //   * merge_b_kernel     the same decomposition on the CUDA cores, for fp32
 //     W_KV (and bf16 shapes the other two do not take).
 // Each is a programmatic dependent of the split kernel: what does not depend
