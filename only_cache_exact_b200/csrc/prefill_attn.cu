@@ -10,24 +10,26 @@
 //     o_i = softmax(q_i · K_{<=p_i}^T / sqrt(d_h)) · V_{<=p_i}
 // per head, p_i the position of query i (its own key included).
 //
-// This kernel is the attention part, flash-attention style on tcgen05 tensor cores: a CTA owns
-// 128 queries of one head of one sequence and walks the 64-key tiles up to its last query's
-// position.
-//   warp 0     TMA producer: the Q tile once, then K and V tiles (64 rows x d_h, 128-byte swizzle,
-//              K and V on separate barriers) through a ring of 5 (d_h = 128) or 8 stages
-//   warp 1     tcgen05.mma issuer: S = Q·K^T (M = 128 queries, N = 64 keys, K = d_h) into one of
-//              two 64-column TMEM buffers, so that the next tile's scores are computed while this
-//              tile's softmax runs; O += P·V (M = 128, N = d_h, K = 64 keys) into a third TMEM
-//              region, P read from one of two shared-memory buffers (K-major; the softmax of the
-//              next tile writes the other while this P·V runs) and V in place as the MN-major
-//              operand
-//   warps 4-7  softmax, one query row per thread (TMEM lane = row): the tile's scores, the causal
-//              mask, a running max kept lazily (O is rescaled in TMEM only when a row's max grows by
-//              more than 2^8, so P <= 2^8 stays exact enough in bf16), P in bf16 to shared memory,
-//              the row sums in fp32 registers; at the end o = O / l to global memory.
+// This kernel is the attention part, flash-attention style on tcgen05 tensor cores: a CTA owns two
+// adjacent 128-query tiles of one head of one sequence and walks the 64-key tiles up to its last
+// query's position; every K and V tile it loads serves both query tiles.
+//   warp 0     TMA producer: the two Q tiles once, then K and V tiles (64 rows x d_h, 128-byte
+//              swizzle, K and V on separate barriers) through a ring of 3 (d_h = 128) or 8 stages
+//   warp 1     tcgen05.mma issuer, per query tile t: S_t = Q_t·K^T (M = 128 queries, N = 64 keys,
+//              K = d_h) into one of two 64-column TMEM buffers of the tile; O_t += P_t·V (M = 128,
+//              N = d_h, K = 64 keys) into the tile's O region, P_t read from one of two
+//              shared-memory buffers of the tile (K-major) and V in place as the MN-major operand.
+//              Issue order S_0(j+1), O_0 += P_0(j)·V_j, S_1(j+1), O_1 += P_1(j)·V_j: while one tile's
+//              softmax of key tile j runs, the tensor cores work through the other tile's MMAs, so a
+//              softmax has four MMA blocks' time instead of two.
+//   warps 2-5  softmax of query tile 0, warps 6-9 of query tile 1, one query row per thread (TMEM
+//              lane = row; warp w reads lanes 32 (w mod 4) ..): the tile's scores, the causal mask, a
+//              running max kept lazily (O is rescaled in TMEM only when a row's max grows by more
+//              than 2^8, so P <= 2^8 stays exact enough in bf16), P in bf16 to shared memory, the row
+//              sums in fp32 registers; at the end o = O / l to global memory.
 // Key rows at or past a sequence's length are scratch in the V buffer: their rows of the last
-// tile are zeroed in shared memory before the P·V MMA (a masked score's p = 0 never meets a
-// non-finite value).
+// tile are zeroed in shared memory before the first P·V MMA that reads them (a masked score's
+// p = 0 never meets a non-finite value).
 #include <cuda_bf16.h>
 
 #include "ptx.cuh"
@@ -36,9 +38,11 @@ namespace slim {
 
 namespace {
 
-constexpr int kPQ = 128;  // queries per CTA (the MMA's M)
+constexpr int kPQ = 128;  // queries per query tile (the MMA's M)
 constexpr int kPK = 64;   // keys per tile
-constexpr int kPThreads = 256;
+constexpr int kPT = 2;    // query tiles per CTA
+constexpr int kPThreads = 64 + 128 * kPT;  // producer warp, MMA warp, a softmax warpgroup per query tile
+constexpr uint32_t kPTmemPerTile = 256;    // S buffers at columns 0 and 64, O at 128
 constexpr float kPLazyLog2 = 8.f;
 
 struct PrefillAttnParams {
@@ -50,7 +54,7 @@ struct PrefillAttnParams {
   float scale_log2;
 };
 
-__host__ __device__ inline int pa_stages(int dhb) { return dhb == 2 ? 4 : 8; }
+__host__ __device__ inline int pa_stages(int dhb) { return dhb == 2 ? 3 : 8; }
 
 // 2^x on the special-function unit (the PTX approximate base-2 exponential; subnormal results flush
 // to zero, which for a softmax weight below 2^-126 is a zero weight).
@@ -62,8 +66,9 @@ __device__ __forceinline__ float ex2_approx(float x) {
 __host__ __device__ inline uint32_t pa_q_bytes(int dhb) { return 128u * 128u * dhb; }  // 128 queries x d_h bf16
 __host__ __device__ inline uint32_t pa_kv_bytes(int dhb) { return 64u * 128u * dhb; }  // 64 keys x d_h bf16
 __host__ __device__ inline uint32_t pa_smem_bytes(int dhb) {
-  // Q, the K/V ring, two P buffers (128 x 64 bf16), barriers, TMEM slot; slack for 1024-byte alignment
-  return pa_q_bytes(dhb) + pa_stages(dhb) * 2u * pa_kv_bytes(dhb) + 2u * 16384u + 512u + 1024u;
+  // the Q tiles, the K/V ring, two P buffers (128 x 64 bf16) per query tile, barriers, TMEM slot;
+  // slack for 1024-byte alignment
+  return kPT * pa_q_bytes(dhb) + pa_stages(dhb) * 2u * pa_kv_bytes(dhb) + kPT * 2u * 16384u + 512u + 1024u;
 }
 
 template <int DHB>
@@ -73,38 +78,43 @@ __global__ void __launch_bounds__(kPThreads, 1)
   extern __shared__ uint8_t pa_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pa_raw) + 1023) & ~uintptr_t(1023));
   constexpr int DH = 64 * DHB;
-  constexpr int NS = DHB == 2 ? 4 : 8;
+  constexpr int NS = DHB == 2 ? 3 : 8;
   const uint32_t TQ = pa_q_bytes(DHB), T = pa_kv_bytes(DHB);
-  uint8_t* qs = sm;  // [DHB boxes][128 rows][128 B]
-  uint8_t* kvs = sm + TQ;  // [stage][K tile, V tile], each [DHB boxes][64 rows][128 B]
-  uint8_t* ps = sm + TQ + NS * 2u * T;  // P: [2 buffers][128 rows][128 B] (64 keys)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ps + 2u * 16384u);
-  uint64_t* qbar = bars;                // Q landed
-  uint64_t* kfull = bars + 1;           // [NS] K of a tile landed
-  uint64_t* vfull = kfull + NS;         // [NS] V of a tile landed
-  uint64_t* kvempty = vfull + NS;       // [NS] the tile's MMAs are done with the stage
-  uint64_t* sfull = kvempty + NS;       // [2] S buffer written
-  uint64_t* sfree = sfull + 2;          // [2] S buffer read by the four softmax warps
-  uint64_t* pready = sfree + 2;         // [2] P buffer written (and O rescaled) by the four softmax warps
-  uint64_t* pfree = pready + 2;         // [2] the P·V MMA that read the buffer completed
-  uint64_t* ofull = pfree + 2;          // the last P·V MMA completed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ofull + 1);
+  uint8_t* qs = sm;                     // [query tile][DHB boxes][128 rows][128 B]
+  uint8_t* kvs = sm + kPT * TQ;         // [stage][K tile, V tile], each [DHB boxes][64 rows][128 B]
+  uint8_t* ps = kvs + NS * 2u * T;      // P: [query tile][2 buffers][128 rows][128 B] (64 keys)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ps + kPT * 2u * 16384u);
+  uint64_t* qbar = bars;                // the Q tiles landed
+  uint64_t* kfull = bars + 1;           // [NS] K of a key tile landed
+  uint64_t* vfull = kfull + NS;         // [NS] V of a key tile landed
+  uint64_t* kvempty = vfull + NS;       // [NS] the key tile's MMAs are done with the stage
+  uint64_t* sfull = kvempty + NS;       // [query tile][2] S buffer written
+  uint64_t* sfree = sfull + 2 * kPT;    // [query tile][2] S buffer read by the tile's four softmax warps
+  uint64_t* pready = sfree + 2 * kPT;   // [query tile][2] P buffer written (and O rescaled) by the four warps
+  uint64_t* pfree = pready + 2 * kPT;   // [query tile][2] the P·V MMA that read the buffer completed
+  uint64_t* ofull = pfree + 2 * kPT;    // [query tile] the tile's last P·V MMA completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ofull + kPT);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // heaviest query tiles (the last ones) first
+  // heaviest query tiles (the last ones) first; the CTA's tiles are nqt - kPT (pair + 1) + t, a
+  // negative index is an absent tile (an odd number of tiles)
   const int nqt = (p.n + kPQ - 1) / kPQ;
   const int bh = blockIdx.x % (p.B * p.H);
-  const int qt = nqt - 1 - blockIdx.x / (p.B * p.H);
+  const int pair = blockIdx.x / (p.B * p.H);
   const int b = bh / p.H, h = bh - b * p.H;
-  const int q0 = qt * kPQ;
   const int L = __ldg(p.lens + b);
   const int pos0 = L - p.n;  // position of query 0
   if (pos0 < 0 || static_cast<int64_t>(L) > p.cap) {
-    if (threadIdx.x == 0 && h == 0 && qt == 0) atomicOr(p.status, SLIM_DEV_BADLEN);
+    if (threadIdx.x == 0 && h == 0 && pair == 0) atomicOr(p.status, SLIM_DEV_BADLEN);
     return;
   }
-  const int last_key = pos0 + min(q0 + kPQ, p.n) - 1;  // largest position any query here attends
-  const int nkt = last_key / kPK + 1;
+  auto tile_q0 = [&](int t) { return (nqt - kPT * (pair + 1) + t) * kPQ; };
+  // key tiles query tile t attends: up to its last query's position; 0 for an absent tile
+  auto tile_keys = [&](int t) {
+    const int q0 = tile_q0(t);
+    return q0 < 0 ? 0 : (pos0 + min(q0 + kPQ, p.n) - 1) / kPK + 1;
+  };
+  const int nkt = tile_keys(kPT - 1);  // the last tile attends the most keys
 
   if (warp == 0 && lane == 0) {
     mbar_init(qbar, 1);
@@ -113,25 +123,22 @@ __global__ void __launch_bounds__(kPThreads, 1)
       mbar_init(&vfull[s], 1);
       mbar_init(&kvempty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 2 * kPT; ++i) {
       mbar_init(&sfull[i], 1);
       mbar_init(&sfree[i], 4);
-    }
-    for (int i = 0; i < 2; ++i) {
       mbar_init(&pready[i], 4);
       mbar_init(&pfree[i], 1);
     }
-    mbar_init(ofull, 1);
+    for (int t = 0; t < kPT; ++t) mbar_init(&ofull[t], 1);
     fence_barrier_init();
   } else if (warp == 1) {
-    tmem_alloc(tmem_slot, 256);
+    tmem_alloc(tmem_slot, kPTmemPerTile * kPT);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_o = tmem + 128u;  // S buffers at columns 0 and 64
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -139,10 +146,19 @@ __global__ void __launch_bounds__(kPThreads, 1)
       tma_prefetch_desc(&qmap);
       tma_prefetch_desc(&kmap);
       tma_prefetch_desc(&vmap);
-      mbar_arrive_expect_tx(qbar, TQ);
+      uint32_t qbytes = 0;
 #pragma unroll
-      for (int i = 0; i < DHB; ++i)
-        tma_load_2d(qs + i * 16384, &qmap, h * DH + 64 * i, b * p.n + q0, qbar, l2_policy_evict_first());
+      for (int t = 0; t < kPT; ++t)
+        if (tile_keys(t) > 0) qbytes += TQ;
+      mbar_arrive_expect_tx(qbar, qbytes);
+#pragma unroll
+      for (int t = 0; t < kPT; ++t) {
+        if (tile_keys(t) == 0) continue;
+#pragma unroll
+        for (int i = 0; i < DHB; ++i)
+          tma_load_2d(qs + t * TQ + i * 16384, &qmap, h * DH + 64 * i, b * p.n + tile_q0(t), qbar,
+                      l2_policy_evict_first());
+      }
       int j = 0;
       for (; j < nkt; ++j) {
         const int s = j % NS;
@@ -171,62 +187,95 @@ __global__ void __launch_bounds__(kPThreads, 1)
       const uint32_t idesc_s = idesc_bf16_f32(kPQ, kPK, 0u, 0u);
       const uint32_t idesc_o = idesc_bf16_f32(kPQ, DH, 0u, 1u);
       const uint32_t qb = smem_u32(qs), kvb = smem_u32(kvs), pb = smem_u32(ps);
+      int nk[kPT];
+#pragma unroll
+      for (int t = 0; t < kPT; ++t) nk[t] = tile_keys(t);
       bool ok = mbar_wait(qbar, 0u, p.status);
-      auto issue_s = [&](int j) {
+      // S_t(j) = Q_t·K_j^T into the tile's S buffer j mod 2
+      auto issue_s = [&](int t, int j) {
         const int s = j % NS, sb = j & 1;
         if (!mbar_wait(&kfull[s], static_cast<uint32_t>(j / NS) & 1u, p.status)) return false;
-        if (j >= 2 && !mbar_wait(&sfree[sb], static_cast<uint32_t>((j - 2) / 2) & 1u, p.status)) return false;
+        if (j >= 2 && !mbar_wait(&sfree[2 * t + sb], static_cast<uint32_t>((j - 2) / 2) & 1u, p.status))
+          return false;
         tc_fence_after();
-        const uint32_t kb = kvb + s * 2u * T;
+        const uint32_t kb = kvb + s * 2u * T, qtb = qb + t * TQ;
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk) {
           // Q and K both K-major (d_h contiguous): 64-column boxes 16 KB (Q) or 8 KB (K) apart, 8-row
           // groups 1024 B apart, a 16-column step is 32 B into the swizzled row
           const uint32_t cin = (kk & 3) * 32u;
-          umma_f16(tmem + static_cast<uint32_t>(sb * kPK),
-                   smem_desc(qb + (kk >> 2) * 16384u + cin, 16, 1024, kLayoutSW128),
+          umma_f16(tmem + t * kPTmemPerTile + static_cast<uint32_t>(sb * kPK),
+                   smem_desc(qtb + (kk >> 2) * 16384u + cin, 16, 1024, kLayoutSW128),
                    smem_desc(kb + (kk >> 2) * 8192u + cin, 16, 1024, kLayoutSW128), idesc_s, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&sfull[sb]);
+        umma_commit(&sfull[2 * t + sb]);
         return true;
       };
-      if (ok) ok = issue_s(0);
-      for (int j = 0; ok && j < nkt; ++j) {
-        if (j + 1 < nkt && !issue_s(j + 1)) {
-          ok = false;
-          break;
-        }
-        if (!mbar_wait(&pready[j & 1], static_cast<uint32_t>(j / 2) & 1u, p.status) ||
-            !mbar_wait(&vfull[j % NS], static_cast<uint32_t>(j / NS) & 1u, p.status)) {
-          ok = false;
-          break;
-        }
+      // O_t += P_t(j)·V_j
+      auto issue_pv = [&](int t, int j) {
+        const int pbuf = j & 1;
+        if (!mbar_wait(&pready[2 * t + pbuf], static_cast<uint32_t>(j / 2) & 1u, p.status) ||
+            !mbar_wait(&vfull[j % NS], static_cast<uint32_t>(j / NS) & 1u, p.status))
+          return false;
         tc_fence_after();
-        const uint32_t vb = kvb + (j % NS) * 2u * T + T;
+        const uint32_t vb = kvb + (j % NS) * 2u * T + T, pt = pb + (2 * t + pbuf) * 16384u;
 #pragma unroll
         for (int kk = 0; kk < kPK / 16; ++kk) {
           // P K-major (keys contiguous, one 64-key box); V MN-major (d_h contiguous): 64-column
           // blocks 8 KB apart, 8-key groups 1024 B apart, 16 keys per step
-          umma_f16(tmem_o, smem_desc(pb + (j & 1) * 16384u + kk * 32u, 16, 1024, kLayoutSW128),
+          umma_f16(tmem + t * kPTmemPerTile + 128u, smem_desc(pt + kk * 32u, 16, 1024, kLayoutSW128),
                    smem_desc(vb + kk * 2048u, 8192, 1024, kLayoutSW128), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&kvempty[j % NS]);
-        umma_commit(&pfree[j & 1]);
+        umma_commit(&pfree[2 * t + pbuf]);
+        return true;
+      };
+      bool committed[kPT];
+#pragma unroll
+      for (int t = 0; t < kPT; ++t) {
+        committed[t] = false;
+        if (ok && nk[t] > 0) ok = issue_s(t, 0);
       }
-      umma_commit(ofull);  // also after a failure: covers every MMA issued
-      mbar_wait(ofull, 0u, p.status);
+      for (int j = 0; ok && j < nkt; ++j) {
+#pragma unroll
+        for (int t = 0; t < kPT; ++t) {
+          if (!ok || j >= nk[t]) continue;
+          if (j + 1 < nk[t] && !issue_s(t, j + 1)) ok = false;
+          if (ok && !issue_pv(t, j)) ok = false;
+          if (ok && j == nk[t] - 1) {
+            umma_commit(&ofull[t]);
+            committed[t] = true;
+          }
+        }
+        if (ok) umma_commit(&kvempty[j % NS]);  // the last tile's P·V is the key tile's last MMA
+      }
+      // also after a failure: each output barrier covers every MMA issued
+#pragma unroll
+      for (int t = 0; t < kPT; ++t)
+        if (!committed[t]) umma_commit(&ofull[t]);
+#pragma unroll
+      for (int t = 0; t < kPT; ++t) mbar_wait(&ofull[t], 0u, p.status);
     }
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------ softmax warps
+  } else {
+    // ------------------------------------------------------------ softmax warpgroup of query tile t
+    const int t = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // query row of the tile = TMEM lane
     const uint32_t lrow = static_cast<uint32_t>(quarter * 32) << 16;
-    const int pos = pos0 + q0 + r;     // position of this row's query
+    const uint32_t ts = tmem + t * kPTmemPerTile, tmem_o = ts + 128u;
+    const int q0 = tile_q0(t), nkt_t = tile_keys(t);
+    // the lowest tile that attends a key tile zeroes its rows past the length
+    const int nkt_below = t > 0 ? tile_keys(t - 1) : 0;
+    uint64_t* t_sfull = sfull + 2 * t;
+    uint64_t* t_sfree = sfree + 2 * t;
+    uint64_t* t_pready = pready + 2 * t;
+    uint64_t* t_pfree = pfree + 2 * t;
+    uint8_t* pst = ps + t * 2u * 16384u;
+    const int pos = pos0 + q0 + r;  // position of this row's query
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < nkt; ++j) {
+    for (int j = 0; j < nkt_t; ++j) {
       const int sb = j & 1, s = j % NS;
-      if (!__all_sync(0xffffffffu, mbar_wait(&sfull[sb], static_cast<uint32_t>(j / 2) & 1u, p.status))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&t_sfull[sb], static_cast<uint32_t>(j / 2) & 1u, p.status))) {
         ok = false;
         break;
       }
@@ -234,11 +283,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
       float sc[kPK];
 #pragma unroll
       for (int c = 0; c < kPK / 16; ++c)
-        tmem_ld16(tmem + lrow + static_cast<uint32_t>(sb * kPK + 16 * c), *reinterpret_cast<float(*)[16]>(sc + 16 * c));
+        tmem_ld16(ts + lrow + static_cast<uint32_t>(sb * kPK + 16 * c), *reinterpret_cast<float(*)[16]>(sc + 16 * c));
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sfree[sb]);
+      if (lane == 0) mbar_arrive(&t_sfree[sb]);
       // keys past this query masked (only a tile that reaches past the query has any); the scale
       // is applied with the exponent below (max(s)·scale = max(s·scale) for scale > 0)
       const int k0 = j * kPK;
@@ -258,7 +307,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
         m = mt;
         l *= alpha;
       }
-      // P = 2^(s·scale - m) in bf16; the row sum adds the rounded values the MMA sees
+      // P = 2^(s·scale - m) in bf16; the row sum adds the fp32 values before rounding (each differs
+      // from the bf16 the MMA sees by at most 2^-9 relative, so l does too)
       uint32_t pk[kPK / 2];
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
       const float nm = m == -INFINITY ? 0.f : -m;
@@ -267,20 +317,21 @@ __global__ void __launch_bounds__(kPThreads, 1)
         const float a = ex2_approx(fmaf(sc[2 * c], p.scale_log2, nm));
         const float bb = ex2_approx(fmaf(sc[2 * c + 1], p.scale_log2, nm));
         const __nv_bfloat162 hv = __floats2bfloat162_rn(a, bb);
-        const float2 f = __bfloat1622float2(hv);
-        ls[c & 3] += f.x + f.y;
+        ls[c & 3] += a + bb;
         pk[c] = *reinterpret_cast<const uint32_t*>(&hv);
       }
       l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-      // this P buffer was last read by the P·V of tile j - 2
+      // this P buffer was last read by the P·V of key tile j - 2
       const int pbuf = j & 1;
-      if (j >= 2 && !__all_sync(0xffffffffu, mbar_wait(&pfree[pbuf], static_cast<uint32_t>((j - 2) / 2) & 1u, p.status))) {
+      if (j >= 2 &&
+          !__all_sync(0xffffffffu, mbar_wait(&t_pfree[pbuf], static_cast<uint32_t>((j - 2) / 2) & 1u, p.status))) {
         ok = false;
         break;
       }
       if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        // O is rescaled once the previous tile's P·V has completed
-        if (!__all_sync(0xffffffffu, mbar_wait(&pfree[pbuf ^ 1], static_cast<uint32_t>((j - 1) / 2) & 1u, p.status))) {
+        // O is rescaled once the previous key tile's P·V has completed
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(&t_pfree[pbuf ^ 1], static_cast<uint32_t>((j - 1) / 2) & 1u, p.status))) {
           ok = false;
           break;
         }
@@ -299,11 +350,12 @@ __global__ void __launch_bounds__(kPThreads, 1)
 #pragma unroll
       for (int c = 0; c < kPK / 8; ++c) {
         const uint32_t off = static_cast<uint32_t>(pbuf * 16384 + r * 128 + ((c ^ (r & 7)) << 4));
-        *reinterpret_cast<uint4*>(ps + off) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        *reinterpret_cast<uint4*>(pst + off) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       }
-      // key rows at or past the length in this tile hold no value: zero them in V (thread r < 64
-      // takes key row r, once the tile's V has landed)
-      if (k0 + kPK > L && r < kPK && k0 + r >= L) {
+      // key rows at or past the length in this key tile hold no value: zero them in V (thread r < 64
+      // takes key row r, once the tile's V has landed), unless a lower query tile attends this key
+      // tile and zeroed them before its own P·V
+      if (k0 + kPK > L && j >= nkt_below && r < kPK && k0 + r >= L) {
         if (mbar_wait(&vfull[s], static_cast<uint32_t>(j / NS) & 1u, p.status)) {
           uint8_t* vrow = kvs + s * 2u * T + T + r * 128;
 #pragma unroll
@@ -315,22 +367,24 @@ __global__ void __launch_bounds__(kPThreads, 1)
       fence_proxy_async_smem();  // P (and zeroed V rows) are read by the tensor cores
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&pready[pbuf]);
+      if (lane == 0) mbar_arrive(&t_pready[pbuf]);
     }
     // o = O / l
-    const bool got = ok && __all_sync(0xffffffffu, mbar_wait(ofull, 0u, p.status));
-    tc_fence_after();
-    const int qi = q0 + r;
-    const float inv = (got && l > 0.f) ? 1.f / l : 0.f;
-    float* dst = p.out + (static_cast<size_t>(b) * p.n + qi) * p.d + h * DH;
-    for (int c = 0; c < DH; c += 16) {
-      float v[16];
-      tmem_ld16(tmem_o + lrow + static_cast<uint32_t>(c), v);
-      tmem_wait_ld();
-      if (qi < p.n) {
+    if (nkt_t > 0) {
+      const bool got = ok && __all_sync(0xffffffffu, mbar_wait(&ofull[t], 0u, p.status));
+      tc_fence_after();
+      const int qi = q0 + r;
+      const float inv = (got && l > 0.f) ? 1.f / l : 0.f;
+      float* dst = p.out + (static_cast<size_t>(b) * p.n + qi) * p.d + h * DH;
+      for (int c = 0; c < DH; c += 16) {
+        float v[16];
+        tmem_ld16(tmem_o + lrow + static_cast<uint32_t>(c), v);
+        tmem_wait_ld();
+        if (qi < p.n) {
 #pragma unroll
-        for (int i = 0; i < 16; i += 4)
-          *reinterpret_cast<float4*>(dst + c + i) = make_float4(v[i] * inv, v[i + 1] * inv, v[i + 2] * inv, v[i + 3] * inv);
+          for (int i = 0; i < 16; i += 4)
+            *reinterpret_cast<float4*>(dst + c + i) = make_float4(v[i] * inv, v[i + 1] * inv, v[i + 2] * inv, v[i + 3] * inv);
+        }
       }
     }
   }
@@ -339,7 +393,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, kPTmemPerTile * kPT);
   }
 }
 
@@ -377,7 +431,8 @@ cudaError_t launch_prefill_attn(const void* Q, const void* kcache, const void* v
   auto kern = dhb == 1 ? prefill_attn_kernel<1> : prefill_attn_kernel<2>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const unsigned grid = static_cast<unsigned>(B * H * ((n + kPQ - 1) / kPQ));
+  const int nqt = (n + kPQ - 1) / kPQ;
+  const unsigned grid = static_cast<unsigned>(B * H * ((nqt + kPT - 1) / kPT));
   kern<<<grid, kPThreads, smem, st>>>(qmap, kmap, vmap, prm);
   e = cudaGetLastError();
   if (e == cudaSuccess && launches) ++*launches;
