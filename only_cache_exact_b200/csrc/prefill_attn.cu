@@ -14,19 +14,23 @@
 // adjacent 128-query tiles of one head of one sequence and walks the 64-key tiles up to its last
 // query's position; every K and V tile it loads serves both query tiles.
 //   warp 0     TMA producer: the two Q tiles once, then K and V tiles (64 rows x d_h, 128-byte
-//              swizzle, K and V on separate barriers) through a ring of 3 (d_h = 128) or 8 stages
+//              swizzle, K and V on separate barriers) through a ring of 5 (d_h = 128) or 8 stages
 //   warp 1     tcgen05.mma issuer, per query tile t: S_t = Q_t·K^T (M = 128 queries, N = 64 keys,
 //              K = d_h) into one of two 64-column TMEM buffers of the tile; O_t += P_t·V (M = 128,
-//              N = d_h, K = 64 keys) into the tile's O region, P_t read from one of two
-//              shared-memory buffers of the tile (K-major) and V in place as the MN-major operand.
+//              N = d_h, K = 64 keys) into the tile's O region, P_t read from tensor memory (the
+//              first 32 columns of the S buffer it was computed from, bf16 pairs) and V in place
+//              from shared memory as the MN-major operand.
 //              Issue order S_0(j+1), O_0 += P_0(j)·V_j, S_1(j+1), O_1 += P_1(j)·V_j: while one tile's
 //              softmax of key tile j runs, the tensor cores work through the other tile's MMAs, so a
 //              softmax has four MMA blocks' time instead of two.
 //   warps 2-5  softmax of query tile 0, warps 6-9 of query tile 1, one query row per thread (TMEM
 //              lane = row; warp w reads lanes 32 (w mod 4) ..): the tile's scores, the causal mask, a
 //              running max kept lazily (O is rescaled in TMEM only when a row's max grows by more
-//              than 2^8, so P <= 2^8 stays exact enough in bf16), P in bf16 to shared memory, the row
-//              sums in fp32 registers; at the end o = O / l to global memory.
+//              than 2^8, so P <= 2^8 stays exact enough in bf16), P in bf16 over the S buffer's
+//              columns in tensor memory, the row sums in fp32 registers; at the end o = O / l to
+//              global memory.
+// The tensor cores run one CTA's MMAs in issue order, so the S MMA that next writes an S buffer
+// (issued after the P·V MMA that reads the P stored there) never overwrites P before it is read.
 // Key rows at or past a sequence's length are scratch in the V buffer: their rows of the last
 // tile are zeroed in shared memory before the first P·V MMA that reads them (a masked score's
 // p = 0 never meets a non-finite value).
@@ -54,7 +58,7 @@ struct PrefillAttnParams {
   float scale_log2;
 };
 
-__host__ __device__ inline int pa_stages(int dhb) { return dhb == 2 ? 3 : 8; }
+__host__ __device__ inline int pa_stages(int dhb) { return dhb == 2 ? 5 : 8; }
 
 // 2^x on the special-function unit (the PTX approximate base-2 exponential; subnormal results flush
 // to zero, which for a softmax weight below 2^-126 is a zero weight).
@@ -66,9 +70,29 @@ __device__ __forceinline__ float ex2_approx(float x) {
 __host__ __device__ inline uint32_t pa_q_bytes(int dhb) { return 128u * 128u * dhb; }  // 128 queries x d_h bf16
 __host__ __device__ inline uint32_t pa_kv_bytes(int dhb) { return 64u * 128u * dhb; }  // 64 keys x d_h bf16
 __host__ __device__ inline uint32_t pa_smem_bytes(int dhb) {
-  // the Q tiles, the K/V ring, two P buffers (128 x 64 bf16) per query tile, barriers, TMEM slot;
-  // slack for 1024-byte alignment
-  return kPT * pa_q_bytes(dhb) + pa_stages(dhb) * 2u * pa_kv_bytes(dhb) + kPT * 2u * 16384u + 512u + 1024u;
+  // the Q tiles, the K/V ring, barriers, TMEM slot; slack for 1024-byte alignment
+  return kPT * pa_q_bytes(dhb) + pa_stages(dhb) * 2u * pa_kv_bytes(dhb) + 512u + 1024u;
+}
+
+// 16 consecutive 32-bit TMEM columns of this thread's lane (32x32b shape, one lane per thread).
+__device__ __forceinline__ void tmem_st16_u32(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
+// D (TMEM) (+)= A · B with the bf16 A operand in tensor memory (K-major: row i in lane i, two
+// elements per 32-bit column) and B from a shared-memory descriptor.
+__device__ __forceinline__ void umma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
 template <int DHB>
@@ -78,20 +102,19 @@ __global__ void __launch_bounds__(kPThreads, 1)
   extern __shared__ uint8_t pa_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pa_raw) + 1023) & ~uintptr_t(1023));
   constexpr int DH = 64 * DHB;
-  constexpr int NS = DHB == 2 ? 3 : 8;
+  constexpr int NS = DHB == 2 ? 5 : 8;
   const uint32_t TQ = pa_q_bytes(DHB), T = pa_kv_bytes(DHB);
   uint8_t* qs = sm;                     // [query tile][DHB boxes][128 rows][128 B]
   uint8_t* kvs = sm + kPT * TQ;         // [stage][K tile, V tile], each [DHB boxes][64 rows][128 B]
-  uint8_t* ps = kvs + NS * 2u * T;      // P: [query tile][2 buffers][128 rows][128 B] (64 keys)
-  uint64_t* bars = reinterpret_cast<uint64_t*>(ps + kPT * 2u * 16384u);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(kvs + NS * 2u * T);
   uint64_t* qbar = bars;                // the Q tiles landed
   uint64_t* kfull = bars + 1;           // [NS] K of a key tile landed
   uint64_t* vfull = kfull + NS;         // [NS] V of a key tile landed
   uint64_t* kvempty = vfull + NS;       // [NS] the key tile's MMAs are done with the stage
   uint64_t* sfull = kvempty + NS;       // [query tile][2] S buffer written
   uint64_t* sfree = sfull + 2 * kPT;    // [query tile][2] S buffer read by the tile's four softmax warps
-  uint64_t* pready = sfree + 2 * kPT;   // [query tile][2] P buffer written (and O rescaled) by the four warps
-  uint64_t* pfree = pready + 2 * kPT;   // [query tile][2] the P·V MMA that read the buffer completed
+  uint64_t* pready = sfree + 2 * kPT;   // [query tile][2] P written over the S buffer (and O rescaled) by the four warps
+  uint64_t* pfree = pready + 2 * kPT;   // [query tile][2] the P·V MMA that read the buffer's P completed
   uint64_t* ofull = pfree + 2 * kPT;    // [query tile] the tile's last P·V MMA completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ofull + kPT);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -186,7 +209,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(kPQ, kPK, 0u, 0u);
       const uint32_t idesc_o = idesc_bf16_f32(kPQ, DH, 0u, 1u);
-      const uint32_t qb = smem_u32(qs), kvb = smem_u32(kvs), pb = smem_u32(ps);
+      const uint32_t qb = smem_u32(qs), kvb = smem_u32(kvs);
       int nk[kPT];
 #pragma unroll
       for (int t = 0; t < kPT; ++t) nk[t] = tile_keys(t);
@@ -218,13 +241,14 @@ __global__ void __launch_bounds__(kPThreads, 1)
             !mbar_wait(&vfull[j % NS], static_cast<uint32_t>(j / NS) & 1u, p.status))
           return false;
         tc_fence_after();
-        const uint32_t vb = kvb + (j % NS) * 2u * T + T, pt = pb + (2 * t + pbuf) * 16384u;
+        const uint32_t vb = kvb + (j % NS) * 2u * T + T;
+        const uint32_t pt = tmem + t * kPTmemPerTile + static_cast<uint32_t>(pbuf * kPK);
 #pragma unroll
         for (int kk = 0; kk < kPK / 16; ++kk) {
-          // P K-major (keys contiguous, one 64-key box); V MN-major (d_h contiguous): 64-column
-          // blocks 8 KB apart, 8-key groups 1024 B apart, 16 keys per step
-          umma_f16(tmem + t * kPTmemPerTile + 128u, smem_desc(pt + kk * 32u, 16, 1024, kLayoutSW128),
-                   smem_desc(vb + kk * 2048u, 8192, 1024, kLayoutSW128), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+          // P in TMEM, 16 keys = 8 columns per step; V MN-major (d_h contiguous): 64-column blocks
+          // 8 KB apart, 8-key groups 1024 B apart, 16 keys per step
+          umma_f16_tmem_a(tmem + t * kPTmemPerTile + 128u, pt + static_cast<uint32_t>(kk * 8),
+                          smem_desc(vb + kk * 2048u, 8192, 1024, kLayoutSW128), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&pfree[2 * t + pbuf]);
         return true;
@@ -269,7 +293,6 @@ __global__ void __launch_bounds__(kPThreads, 1)
     uint64_t* t_sfree = sfree + 2 * t;
     uint64_t* t_pready = pready + 2 * t;
     uint64_t* t_pfree = pfree + 2 * t;
-    uint8_t* pst = ps + t * 2u * 16384u;
     const int pos = pos0 + q0 + r;  // position of this row's query
     float m = -INFINITY, l = 0.f;
     bool ok = true;
@@ -321,13 +344,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
         pk[c] = *reinterpret_cast<const uint32_t*>(&hv);
       }
       l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-      // this P buffer was last read by the P·V of key tile j - 2
+      // P goes over this S buffer: the P·V of key tile j - 2, which read the buffer's previous P,
+      // ran before the S MMA that wrote S(j) there
       const int pbuf = j & 1;
-      if (j >= 2 &&
-          !__all_sync(0xffffffffu, mbar_wait(&t_pfree[pbuf], static_cast<uint32_t>((j - 2) / 2) & 1u, p.status))) {
-        ok = false;
-        break;
-      }
       if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
         // O is rescaled once the previous key tile's P·V has completed
         if (!__all_sync(0xffffffffu,
@@ -346,12 +365,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
         }
         tmem_wait_st();
       }
-      // P row r: [row][16-byte chunk ^ (row & 7)]
-#pragma unroll
-      for (int c = 0; c < kPK / 8; ++c) {
-        const uint32_t off = static_cast<uint32_t>(pbuf * 16384 + r * 128 + ((c ^ (r & 7)) << 4));
-        *reinterpret_cast<uint4*>(pst + off) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      }
+      // P row r: keys 2c, 2c + 1 in column c of the row's lane
+      tmem_st16_u32(ts + lrow + static_cast<uint32_t>(sb * kPK), pk);
+      tmem_st16_u32(ts + lrow + static_cast<uint32_t>(sb * kPK + 16), pk + 16);
+      tmem_wait_st();
       // key rows at or past the length in this key tile hold no value: zero them in V (thread r < 64
       // takes key row r, once the tile's V has landed), unless a lower query tile attends this key
       // tile and zeroed them before its own P·V
@@ -364,7 +381,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
             for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(vrow + i * 8192 + c * 16) = make_uint4(0u, 0u, 0u, 0u);
         }
       }
-      fence_proxy_async_smem();  // P (and zeroed V rows) are read by the tensor cores
+      fence_proxy_async_smem();  // zeroed V rows are read by the tensor cores
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&t_pready[pbuf]);
