@@ -11,26 +11,25 @@
 // per head, p_i the position of query i (its own key included).
 //
 // This kernel is the attention part, flash-attention style on tcgen05 tensor cores: a CTA owns two
-// adjacent 128-query tiles of one head of one sequence and walks the 64-key tiles up to its last
+// adjacent 128-query tiles of one head of one sequence and walks the 128-key tiles up to its last
 // query's position; every K and V tile it loads serves both query tiles.
-//   warp 0     TMA producer: the two Q tiles once, then K and V tiles (64 rows x d_h, 128-byte
-//              swizzle, K and V on separate barriers) through a ring of 5 (d_h = 128) or 8 stages
-//   warp 1     tcgen05.mma issuer, per query tile t: S_t = Q_t·K^T (M = 128 queries, N = 64 keys,
-//              K = d_h) into one of two 64-column TMEM buffers of the tile; O_t += P_t·V (M = 128,
-//              N = d_h, K = 64 keys) into the tile's O region, P_t read from tensor memory (the
-//              first 32 columns of the S buffer it was computed from, bf16 pairs) and V in place
-//              from shared memory as the MN-major operand.
-//              Issue order S_0(j+1), O_0 += P_0(j)·V_j, S_1(j+1), O_1 += P_1(j)·V_j: while one tile's
-//              softmax of key tile j runs, the tensor cores work through the other tile's MMAs, so a
-//              softmax has four MMA blocks' time instead of two.
+//   warp 0     TMA producer: the two Q tiles once, then K and V tiles (128 rows x d_h, 128-byte
+//              swizzle) through separate K and V rings of 2 (d_h = 128) or 6 stages; a K stage is
+//              released when the last S MMA that reads it completes, a V stage with the last P·V
+//   warp 1     tcgen05.mma issuer, per query tile t: S_t = Q_t·K^T (M = 128 queries, N = 128 keys,
+//              K = d_h) into the tile's 128-column TMEM S region; O_t += P_t·V (M = 128, N = d_h,
+//              K = 128 keys) into the tile's O region, P_t read from tensor memory (the first 64
+//              columns of the S region, bf16 pairs) and V in place from shared memory as the
+//              MN-major operand. Issue order P_0(j)·V_j, S_0(j+1), P_1(j)·V_j, S_1(j+1): while one
+//              tile's softmax runs, the tensor cores work through the other tile's MMAs.
 //   warps 2-5  softmax of query tile 0, warps 6-9 of query tile 1, one query row per thread (TMEM
 //              lane = row; warp w reads lanes 32 (w mod 4) ..): the tile's scores, the causal mask, a
 //              running max kept lazily (O is rescaled in TMEM only when a row's max grows by more
-//              than 2^8, so P <= 2^8 stays exact enough in bf16), P in bf16 over the S buffer's
-//              columns in tensor memory, the row sums in fp32 registers; at the end o = O / l to
-//              global memory.
-// The tensor cores run one CTA's MMAs in issue order, so the S MMA that next writes an S buffer
-// (issued after the P·V MMA that reads the P stored there) never overwrites P before it is read.
+//              than 2^8, so P <= 2^8 stays exact enough in bf16), P in bf16 over the S region in
+//              tensor memory, the row sums in fp32 registers; at the end o = O / l to global memory.
+// The tensor cores run one CTA's MMAs in issue order, so the S MMA that next writes a tile's S
+// region (issued after the P·V MMA that reads the P stored there) never overwrites P before it is
+// read.
 // Key rows at or past a sequence's length are scratch in the V buffer: their rows of the last
 // tile are zeroed in shared memory before the first P·V MMA that reads them (a masked score's
 // p = 0 never meets a non-finite value).
@@ -43,10 +42,10 @@ namespace slim {
 namespace {
 
 constexpr int kPQ = 128;  // queries per query tile (the MMA's M)
-constexpr int kPK = 64;   // keys per tile
+constexpr int kPK = 128;  // keys per key tile (the S MMA's N)
 constexpr int kPT = 2;    // query tiles per CTA
 constexpr int kPThreads = 64 + 128 * kPT;  // producer warp, MMA warp, a softmax warpgroup per query tile
-constexpr uint32_t kPTmemPerTile = 256;    // S buffers at columns 0 and 64, O at 128
+constexpr uint32_t kPTmemPerTile = 256;    // S (and P over it) at columns 0..127, O at 128
 constexpr float kPLazyLog2 = 8.f;
 
 struct PrefillAttnParams {
@@ -58,7 +57,7 @@ struct PrefillAttnParams {
   float scale_log2;
 };
 
-__host__ __device__ inline int pa_stages(int dhb) { return dhb == 2 ? 5 : 8; }
+__host__ __device__ inline int pa_stages(int dhb) { return dhb == 2 ? 2 : 6; }
 
 // 2^x on the special-function unit (the PTX approximate base-2 exponential; subnormal results flush
 // to zero, which for a softmax weight below 2^-126 is a zero weight).
@@ -67,10 +66,10 @@ __device__ __forceinline__ float ex2_approx(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-__host__ __device__ inline uint32_t pa_q_bytes(int dhb) { return 128u * 128u * dhb; }  // 128 queries x d_h bf16
-__host__ __device__ inline uint32_t pa_kv_bytes(int dhb) { return 64u * 128u * dhb; }  // 64 keys x d_h bf16
+__host__ __device__ inline uint32_t pa_q_bytes(int dhb) { return 128u * 128u * dhb; }   // 128 queries x d_h bf16
+__host__ __device__ inline uint32_t pa_kv_bytes(int dhb) { return 128u * 128u * dhb; }  // 128 keys x d_h bf16
 __host__ __device__ inline uint32_t pa_smem_bytes(int dhb) {
-  // the Q tiles, the K/V ring, barriers, TMEM slot; slack for 1024-byte alignment
+  // the Q tiles, the K and V rings, barriers, TMEM slot; slack for 1024-byte alignment
   return kPT * pa_q_bytes(dhb) + pa_stages(dhb) * 2u * pa_kv_bytes(dhb) + 512u + 1024u;
 }
 
@@ -102,20 +101,21 @@ __global__ void __launch_bounds__(kPThreads, 1)
   extern __shared__ uint8_t pa_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pa_raw) + 1023) & ~uintptr_t(1023));
   constexpr int DH = 64 * DHB;
-  constexpr int NS = DHB == 2 ? 5 : 8;
+  constexpr int NS = DHB == 2 ? 2 : 6;
   const uint32_t TQ = pa_q_bytes(DHB), T = pa_kv_bytes(DHB);
-  uint8_t* qs = sm;                     // [query tile][DHB boxes][128 rows][128 B]
-  uint8_t* kvs = sm + kPT * TQ;         // [stage][K tile, V tile], each [DHB boxes][64 rows][128 B]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(kvs + NS * 2u * T);
-  uint64_t* qbar = bars;                // the Q tiles landed
-  uint64_t* kfull = bars + 1;           // [NS] K of a key tile landed
-  uint64_t* vfull = kfull + NS;         // [NS] V of a key tile landed
-  uint64_t* kvempty = vfull + NS;       // [NS] the key tile's MMAs are done with the stage
-  uint64_t* sfull = kvempty + NS;       // [query tile][2] S buffer written
-  uint64_t* sfree = sfull + 2 * kPT;    // [query tile][2] S buffer read by the tile's four softmax warps
-  uint64_t* pready = sfree + 2 * kPT;   // [query tile][2] P written over the S buffer (and O rescaled) by the four warps
-  uint64_t* pfree = pready + 2 * kPT;   // [query tile][2] the P·V MMA that read the buffer's P completed
-  uint64_t* ofull = pfree + 2 * kPT;    // [query tile] the tile's last P·V MMA completed
+  uint8_t* qs = sm;                // [query tile][DHB boxes][128 rows][128 B]
+  uint8_t* ks = sm + kPT * TQ;     // K ring: [stage][DHB boxes][128 rows][128 B]
+  uint8_t* vs = ks + NS * T;       // V ring: [stage][DHB boxes][128 rows][128 B]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(vs + NS * T);
+  uint64_t* qbar = bars;           // the Q tiles landed
+  uint64_t* kfull = bars + 1;      // [NS] K of a key tile landed
+  uint64_t* kempty = kfull + NS;   // [NS] the key tile's S MMAs completed
+  uint64_t* vfull = kempty + NS;   // [NS] V of a key tile landed
+  uint64_t* vempty = vfull + NS;   // [NS] the key tile's P·V MMAs completed
+  uint64_t* sfull = vempty + NS;   // [query tile] S written
+  uint64_t* pready = sfull + kPT;  // [query tile] S read, P written over it (and O rescaled) by the four warps
+  uint64_t* pfree = pready + kPT;  // [query tile] the P·V MMA completed
+  uint64_t* ofull = pfree + kPT;   // [query tile] the tile's last P·V MMA completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ofull + kPT);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -143,16 +143,16 @@ __global__ void __launch_bounds__(kPThreads, 1)
     mbar_init(qbar, 1);
     for (int s = 0; s < NS; ++s) {
       mbar_init(&kfull[s], 1);
+      mbar_init(&kempty[s], 1);
       mbar_init(&vfull[s], 1);
-      mbar_init(&kvempty[s], 1);
+      mbar_init(&vempty[s], 1);
     }
-    for (int i = 0; i < 2 * kPT; ++i) {
-      mbar_init(&sfull[i], 1);
-      mbar_init(&sfree[i], 4);
-      mbar_init(&pready[i], 4);
-      mbar_init(&pfree[i], 1);
+    for (int t = 0; t < kPT; ++t) {
+      mbar_init(&sfull[t], 1);
+      mbar_init(&pready[t], 4);
+      mbar_init(&pfree[t], 1);
+      mbar_init(&ofull[t], 1);
     }
-    for (int t = 0; t < kPT; ++t) mbar_init(&ofull[t], 1);
     fence_barrier_init();
   } else if (warp == 1) {
     tmem_alloc(tmem_slot, kPTmemPerTile * kPT);
@@ -182,75 +182,76 @@ __global__ void __launch_bounds__(kPThreads, 1)
           tma_load_2d(qs + t * TQ + i * 16384, &qmap, h * DH + 64 * i, b * p.n + tile_q0(t), qbar,
                       l2_policy_evict_first());
       }
-      int j = 0;
-      for (; j < nkt; ++j) {
+      int nk_issued = 0, nv_issued = 0;
+      for (int j = 0; j < nkt; ++j) {
         const int s = j % NS;
-        if (j >= NS && !mbar_wait(&kvempty[s], static_cast<uint32_t>((j / NS) & 1) ^ 1u, p.status)) break;
-        uint8_t* dst = kvs + s * 2u * T;
+        const uint32_t ph = static_cast<uint32_t>((j / NS) & 1);
         const int y = static_cast<int>(static_cast<int64_t>(b) * p.cap + j * kPK);
+        if (j >= NS && !mbar_wait(&kempty[s], ph ^ 1u, p.status)) break;
         mbar_arrive_expect_tx(&kfull[s], T);
 #pragma unroll
         for (int i = 0; i < DHB; ++i)
-          tma_load_2d(dst + i * 8192, &kmap, h * DH + 64 * i, y, &kfull[s], l2_policy_evict_last());
+          tma_load_2d(ks + s * T + i * 16384, &kmap, h * DH + 64 * i, y, &kfull[s], l2_policy_evict_last());
+        ++nk_issued;
+        if (j >= NS && !mbar_wait(&vempty[s], ph ^ 1u, p.status)) break;
         mbar_arrive_expect_tx(&vfull[s], T);
 #pragma unroll
         for (int i = 0; i < DHB; ++i)
-          tma_load_2d(dst + T + i * 8192, &vmap, h * DH + 64 * i, y, &vfull[s], l2_policy_evict_last());
+          tma_load_2d(vs + s * T + i * 16384, &vmap, h * DH + 64 * i, y, &vfull[s], l2_policy_evict_last());
+        ++nv_issued;
       }
       // every issued copy lands before the CTA exits
       mbar_wait(qbar, 0u, p.status);
-      for (int t = max(0, j - NS); t < j; ++t) {
-        mbar_wait(&kfull[t % NS], static_cast<uint32_t>(t / NS) & 1u, p.status);
-        mbar_wait(&vfull[t % NS], static_cast<uint32_t>(t / NS) & 1u, p.status);
-      }
+      for (int u = max(0, nk_issued - NS); u < nk_issued; ++u)
+        mbar_wait(&kfull[u % NS], static_cast<uint32_t>(u / NS) & 1u, p.status);
+      for (int u = max(0, nv_issued - NS); u < nv_issued; ++u)
+        mbar_wait(&vfull[u % NS], static_cast<uint32_t>(u / NS) & 1u, p.status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(kPQ, kPK, 0u, 0u);
       const uint32_t idesc_o = idesc_bf16_f32(kPQ, DH, 0u, 1u);
-      const uint32_t qb = smem_u32(qs), kvb = smem_u32(kvs);
+      const uint32_t qb = smem_u32(qs), kb0 = smem_u32(ks), vb0 = smem_u32(vs);
       int nk[kPT];
 #pragma unroll
       for (int t = 0; t < kPT; ++t) nk[t] = tile_keys(t);
       bool ok = mbar_wait(qbar, 0u, p.status);
-      // S_t(j) = Q_t·K_j^T into the tile's S buffer j mod 2
+      // S_t(j) = Q_t·K_j^T into the tile's S region; the last tile's S MMA is the last reader of K_j
       auto issue_s = [&](int t, int j) {
-        const int s = j % NS, sb = j & 1;
+        const int s = j % NS;
         if (!mbar_wait(&kfull[s], static_cast<uint32_t>(j / NS) & 1u, p.status)) return false;
-        if (j >= 2 && !mbar_wait(&sfree[2 * t + sb], static_cast<uint32_t>((j - 2) / 2) & 1u, p.status))
-          return false;
         tc_fence_after();
-        const uint32_t kb = kvb + s * 2u * T, qtb = qb + t * TQ;
+        const uint32_t kb = kb0 + s * T, qtb = qb + t * TQ;
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk) {
-          // Q and K both K-major (d_h contiguous): 64-column boxes 16 KB (Q) or 8 KB (K) apart, 8-row
-          // groups 1024 B apart, a 16-column step is 32 B into the swizzled row
-          const uint32_t cin = (kk & 3) * 32u;
-          umma_f16(tmem + t * kPTmemPerTile + static_cast<uint32_t>(sb * kPK),
-                   smem_desc(qtb + (kk >> 2) * 16384u + cin, 16, 1024, kLayoutSW128),
-                   smem_desc(kb + (kk >> 2) * 8192u + cin, 16, 1024, kLayoutSW128), idesc_s, kk > 0 ? 1u : 0u);
+          // Q and K both K-major (d_h contiguous): 64-column boxes 16 KB apart, 8-row groups 1024 B
+          // apart, a 16-column step is 32 B into the swizzled row
+          const uint32_t off = (kk >> 2) * 16384u + (kk & 3) * 32u;
+          umma_f16(tmem + t * kPTmemPerTile, smem_desc(qtb + off, 16, 1024, kLayoutSW128),
+                   smem_desc(kb + off, 16, 1024, kLayoutSW128), idesc_s, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&sfull[2 * t + sb]);
+        umma_commit(&sfull[t]);
+        if (t == kPT - 1) umma_commit(&kempty[s]);
         return true;
       };
-      // O_t += P_t(j)·V_j
+      // O_t += P_t(j)·V_j; the last tile's P·V is the last reader of V_j
       auto issue_pv = [&](int t, int j) {
-        const int pbuf = j & 1;
-        if (!mbar_wait(&pready[2 * t + pbuf], static_cast<uint32_t>(j / 2) & 1u, p.status) ||
-            !mbar_wait(&vfull[j % NS], static_cast<uint32_t>(j / NS) & 1u, p.status))
+        const int s = j % NS;
+        if (!mbar_wait(&pready[t], static_cast<uint32_t>(j) & 1u, p.status) ||
+            !mbar_wait(&vfull[s], static_cast<uint32_t>(j / NS) & 1u, p.status))
           return false;
         tc_fence_after();
-        const uint32_t vb = kvb + (j % NS) * 2u * T + T;
-        const uint32_t pt = tmem + t * kPTmemPerTile + static_cast<uint32_t>(pbuf * kPK);
+        const uint32_t vb = vb0 + s * T, pt = tmem + t * kPTmemPerTile;
 #pragma unroll
         for (int kk = 0; kk < kPK / 16; ++kk) {
           // P in TMEM, 16 keys = 8 columns per step; V MN-major (d_h contiguous): 64-column blocks
-          // 8 KB apart, 8-key groups 1024 B apart, 16 keys per step
+          // 16 KB apart, 8-key groups 1024 B apart, 16 keys per step
           umma_f16_tmem_a(tmem + t * kPTmemPerTile + 128u, pt + static_cast<uint32_t>(kk * 8),
-                          smem_desc(vb + kk * 2048u, 8192, 1024, kLayoutSW128), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                          smem_desc(vb + kk * 2048u, 16384, 1024, kLayoutSW128), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&pfree[2 * t + pbuf]);
+        umma_commit(&pfree[t]);
+        if (t == kPT - 1) umma_commit(&vempty[s]);
         return true;
       };
       bool committed[kPT];
@@ -263,14 +264,14 @@ __global__ void __launch_bounds__(kPThreads, 1)
 #pragma unroll
         for (int t = 0; t < kPT; ++t) {
           if (!ok || j >= nk[t]) continue;
-          if (j + 1 < nk[t] && !issue_s(t, j + 1)) ok = false;
-          if (ok && !issue_pv(t, j)) ok = false;
+          if (!issue_pv(t, j)) ok = false;
           if (ok && j == nk[t] - 1) {
             umma_commit(&ofull[t]);
             committed[t] = true;
           }
+          // S_t(j+1) overwrites the P that the P·V above reads: issued after it
+          if (ok && j + 1 < nk[t] && !issue_s(t, j + 1)) ok = false;
         }
-        if (ok) umma_commit(&kvempty[j % NS]);  // the last tile's P·V is the key tile's last MMA
       }
       // also after a failure: each output barrier covers every MMA issued
 #pragma unroll
@@ -289,16 +290,12 @@ __global__ void __launch_bounds__(kPThreads, 1)
     const int q0 = tile_q0(t), nkt_t = tile_keys(t);
     // the lowest tile that attends a key tile zeroes its rows past the length
     const int nkt_below = t > 0 ? tile_keys(t - 1) : 0;
-    uint64_t* t_sfull = sfull + 2 * t;
-    uint64_t* t_sfree = sfree + 2 * t;
-    uint64_t* t_pready = pready + 2 * t;
-    uint64_t* t_pfree = pfree + 2 * t;
     const int pos = pos0 + q0 + r;  // position of this row's query
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nkt_t; ++j) {
-      const int sb = j & 1, s = j % NS;
-      if (!__all_sync(0xffffffffu, mbar_wait(&t_sfull[sb], static_cast<uint32_t>(j / 2) & 1u, p.status))) {
+      const int s = j % NS;
+      if (!__all_sync(0xffffffffu, mbar_wait(&sfull[t], static_cast<uint32_t>(j) & 1u, p.status))) {
         ok = false;
         break;
       }
@@ -306,11 +303,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
       float sc[kPK];
 #pragma unroll
       for (int c = 0; c < kPK / 16; ++c)
-        tmem_ld16(ts + lrow + static_cast<uint32_t>(sb * kPK + 16 * c), *reinterpret_cast<float(*)[16]>(sc + 16 * c));
+        tmem_ld16(ts + lrow + static_cast<uint32_t>(16 * c), *reinterpret_cast<float(*)[16]>(sc + 16 * c));
       tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&t_sfree[sb]);
       // keys past this query masked (only a tile that reaches past the query has any); the scale
       // is applied with the exponent below (max(s)·scale = max(s·scale) for scale > 0)
       const int k0 = j * kPK;
@@ -330,27 +324,30 @@ __global__ void __launch_bounds__(kPThreads, 1)
         m = mt;
         l *= alpha;
       }
-      // P = 2^(s·scale - m) in bf16; the row sum adds the fp32 values before rounding (each differs
-      // from the bf16 the MMA sees by at most 2^-9 relative, so l does too)
-      uint32_t pk[kPK / 2];
+      // P = 2^(s·scale - m) in bf16 over the S region, 32 keys (16 columns) at a time: keys 2c and
+      // 2c + 1 in column c of the row's lane. The row sum adds the fp32 values before rounding (each
+      // differs from the bf16 the MMA sees by at most 2^-9 relative, so l does too).
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
       const float nm = m == -INFINITY ? 0.f : -m;
 #pragma unroll
-      for (int c = 0; c < kPK / 2; ++c) {
-        const float a = ex2_approx(fmaf(sc[2 * c], p.scale_log2, nm));
-        const float bb = ex2_approx(fmaf(sc[2 * c + 1], p.scale_log2, nm));
-        const __nv_bfloat162 hv = __floats2bfloat162_rn(a, bb);
-        ls[c & 3] += a + bb;
-        pk[c] = *reinterpret_cast<const uint32_t*>(&hv);
+      for (int q = 0; q < kPK / 32; ++q) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const float a = ex2_approx(fmaf(sc[32 * q + 2 * c], p.scale_log2, nm));
+          const float bb = ex2_approx(fmaf(sc[32 * q + 2 * c + 1], p.scale_log2, nm));
+          const __nv_bfloat162 hv = __floats2bfloat162_rn(a, bb);
+          ls[c & 3] += a + bb;
+          pk[c] = *reinterpret_cast<const uint32_t*>(&hv);
+        }
+        tmem_st16_u32(ts + lrow + static_cast<uint32_t>(16 * q), pk);
       }
       l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-      // P goes over this S buffer: the P·V of key tile j - 2, which read the buffer's previous P,
-      // ran before the S MMA that wrote S(j) there
-      const int pbuf = j & 1;
       if (j >= 1 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        // O is rescaled once the previous key tile's P·V has completed
-        if (!__all_sync(0xffffffffu,
-                        mbar_wait(&t_pfree[pbuf ^ 1], static_cast<uint32_t>((j - 1) / 2) & 1u, p.status))) {
+        // O is rescaled once the previous key tile's P·V has completed (after P, so that the scores
+        // are no longer live)
+        if (!__all_sync(0xffffffffu, mbar_wait(&pfree[t], static_cast<uint32_t>(j - 1) & 1u, p.status))) {
+          tmem_wait_st();
           ok = false;
           break;
         }
@@ -363,28 +360,24 @@ __global__ void __launch_bounds__(kPThreads, 1)
           for (int i = 0; i < 16; ++i) v[i] *= alpha;
           tmem_st16(tmem_o + lrow + static_cast<uint32_t>(c), v);
         }
-        tmem_wait_st();
       }
-      // P row r: keys 2c, 2c + 1 in column c of the row's lane
-      tmem_st16_u32(ts + lrow + static_cast<uint32_t>(sb * kPK), pk);
-      tmem_st16_u32(ts + lrow + static_cast<uint32_t>(sb * kPK + 16), pk + 16);
       tmem_wait_st();
-      // key rows at or past the length in this key tile hold no value: zero them in V (thread r < 64
+      // key rows at or past the length in this key tile hold no value: zero them in V (thread r
       // takes key row r, once the tile's V has landed), unless a lower query tile attends this key
       // tile and zeroed them before its own P·V
-      if (k0 + kPK > L && j >= nkt_below && r < kPK && k0 + r >= L) {
+      if (k0 + kPK > L && j >= nkt_below && k0 + r >= L) {
         if (mbar_wait(&vfull[s], static_cast<uint32_t>(j / NS) & 1u, p.status)) {
-          uint8_t* vrow = kvs + s * 2u * T + T + r * 128;
+          uint8_t* vrow = vs + s * T + r * 128;
 #pragma unroll
           for (int i = 0; i < DHB; ++i)
 #pragma unroll
-            for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(vrow + i * 8192 + c * 16) = make_uint4(0u, 0u, 0u, 0u);
+            for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(vrow + i * 16384 + c * 16) = make_uint4(0u, 0u, 0u, 0u);
         }
       }
       fence_proxy_async_smem();  // zeroed V rows are read by the tensor cores
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&t_pready[pbuf]);
+      if (lane == 0) mbar_arrive(&pready[t]);
     }
     // o = O / l
     if (nkt_t > 0) {

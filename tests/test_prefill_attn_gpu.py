@@ -82,13 +82,13 @@ def test_prompt_attention_d4096(S):
 
 def test_prompt_attention_many_key_tiles(S):
     """d_h = 64, 700 prompt rows after 200 cached ones: up to 8 key tiles of 128 per query tile,
-    both S buffers and the K/V ring reused several times, a ragged last key tile."""
+    the S regions and the K and V rings reused several times, a ragged last key tile."""
     _run(S, 1024, 16, [200], 700, seed=53)
 
 
 def test_prompt_attention_query_tiles_share_the_ragged_key_tile(S):
     """d_h = 128, 140 prompt rows after 10 cached ones: the two 128-query tiles a CTA holds both
-    attend key tile 2 (rows 128..191), whose rows from 150 on are past the length; the lower tile
+    attend key tile 1 (rows 128..255), whose rows from 150 on are past the length; the lower tile
     zeroes them for both."""
     _run(S, 4096, 32, [10], 140, seed=54)
 
