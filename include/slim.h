@@ -198,6 +198,9 @@ int slim_decode_step_x(const void* x, const void* W_Q, const void* W_K, void* Kc
  * serialised by the caller.
  */
 #define SLIM_NOALLOC_SCRATCH_BYTES (32 * 1024 * 1024)
+/* The size of that buffer as compiled into this library (SLIM_NOALLOC_SCRATCH_BYTES of the header it
+ * was built with); host-only, needs no device. */
+size_t slim_noalloc_scratch_bytes(void);
 int slim_decode_step_noalloc(const float* q, const void* k_new, void* Kcache, int32_t* lens, const void* W_KV,
                              int dtype, int B, int d, int H, int64_t cap, int variant, int64_t t_hint, float* out,
                              int32_t* dev_status, void* stream);

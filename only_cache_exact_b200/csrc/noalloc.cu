@@ -46,6 +46,8 @@ int scratch_on_current_device(void** addr) {
 
 }  // namespace
 
+extern "C" size_t slim_noalloc_scratch_bytes(void) { return static_cast<size_t>(SLIM_NOALLOC_SCRATCH_BYTES); }
+
 extern "C" int slim_decode_step_noalloc(const float* q, const void* k_new, void* Kcache, int32_t* lens,
                                         const void* W_KV, int dtype, int B, int d, int H, int64_t cap, int variant,
                                         int64_t t_hint, float* out, int32_t* dev_status, void* stream) {

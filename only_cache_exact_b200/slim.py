@@ -30,7 +30,7 @@ EXPORTS = [
     "slim_version", "slim_timing_enable", "slim_timing_read", "slim_decode_step_noalloc",
     "slim_mha_decode_workspace_bytes", "slim_mha_decode_step", "slim_debug_stall_next",
     "slim_prefill_attention_workspace_bytes", "slim_prefill_attention", "slim_project_qk",
-    "slim_decode_step_x_workspace_bytes", "slim_decode_step_x",
+    "slim_decode_step_x_workspace_bytes", "slim_decode_step_x", "slim_noalloc_scratch_bytes",
 ]
 
 _vp, _i32, _i64, _sz, _f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
@@ -64,12 +64,14 @@ _SIGS = {
     "slim_decode_step_x_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32, _i64, _i32]),
     "slim_decode_step_x": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i64, _i32, _i64, _vp, _vp,
                                   _sz, _vp, _vp]),
+    "slim_noalloc_scratch_bytes": (_sz, []),
 }
-SLIM_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
     _fn.restype = _res
     _fn.argtypes = _args
+# the scratch size compiled into the library, read from it rather than restated
+SLIM_NOALLOC_SCRATCH_BYTES = int(_lib.slim_noalloc_scratch_bytes())
 
 _DT = {torch.bfloat16: SLIM_BF16, torch.float32: SLIM_F32}
 
